@@ -1,0 +1,324 @@
+"""Benchmark of the mask-aware attention forward pass (one JSON line on rank 0).
+
+A step is one pass of the whole hot path on one batch: build the tile map from
+the compact mask description (three kernels), then the forward kernel. The
+metric is effective TFLOP/s counting only visible (query, key) pairs, 4*d FLOPs
+each, over the whole job (all ranks). Inputs are seeded N(0,1) bf16 tensors of
+the named workload's shape; they are resident in HBM when timing starts, and L2
+is flushed (a 256 MiB write) between timed steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload doc8k] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); each rank runs an independent
+replica of the workload (the path needs no exchange), so scaling is weak and
+the value is the sum of all ranks' work over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mask_aware_block_mfa_b200 import workloads as W  # noqa: E402
+
+BLOCKS = {  # launch configuration per workload: (block_q, block_k)
+    "tiny_doc_fp32": (128, 64),
+    "doc8k": (64, 128),
+    "shared_question8k": (64, 128),
+    "band16k": (128, 128),
+    "band16k_neg": (128, 128),
+    "doc32k": (64, 128),
+    "blocksel32k": (64, 64),
+}
+METRIC = "effective TFLOP/s (visible pairs only) and % of B200 bf16 tensor peak"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, 1400.0, "fallback"
+
+
+def visible_pairs(mask) -> int:
+    """Visible pairs from the description's own closed forms (host integer arithmetic)."""
+    total = 0
+    for b in range(mask.B):
+        if mask.kind == W.MASK_BAND:
+            pre, nxt = int(mask.pre_tokens), int(mask.next_tokens)
+            i = np.arange(mask.Nq, dtype=np.int64)
+            lo = np.maximum(i - pre, 0)
+            hi = np.minimum(i + nxt, mask.Nk - 1)
+            total += int(np.maximum(hi - lo + 1, 0).sum())
+        elif mask.kind == W.MASK_BLOCKSEL:
+            sel = mask.sel[b, 0]
+            for qb in range(sel.shape[0]):
+                r0, r1 = qb * 64, min(qb * 64 + 64, mask.Nq)
+                for kb in set(int(x) for x in sel[qb] if x >= 0):
+                    c0, c1 = kb * 64, min(kb * 64 + 64, mask.Nk)
+                    i = np.arange(r0, r1)
+                    total += int(np.clip(np.minimum(i + 1, c1) - c0, 0, None).sum())
+        else:  # documents / shared question: the generator's record of the segments
+            if mask.docs is None:
+                raise ValueError("column-wise mask without a segment record")
+            docs = mask.docs[b]
+            if mask.name.startswith("shared_question"):
+                q_len = docs[0][1]
+                total += q_len * (q_len + 1) // 2
+                for (s, e) in docs[1:]:
+                    L = e - s
+                    total += L * q_len + L * (L + 1) // 2
+            else:
+                total += sum((e - s) * (e - s + 1) // 2 for (s, e) in docs)
+    return total
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+        else:
+            self.out = ""
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_reference(args, prob, pairs, d, Hq):
+    """The reference arm: the float64 CPU oracle, each step a bounded sample of the workload."""
+    from threadpoolctl import threadpool_info
+    from oracle import attention as OA
+    heads = list(range(min(args.reference_heads, Hq)))
+    flops = 4.0 * d * pairs * len(heads) / (1 if prob.mask.Hm == 1 else Hq)
+    times = []
+    for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        OA.attention(prob.q, prob.k, prob.v, prob.mask, heads=heads)
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    sec = sum(times) / len(times)
+    value = flops / sec / 1e12
+    return {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.workload, "sample": f"{len(heads)} of {Hq} query heads, all rows"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{len(heads)} of {Hq} query heads, all rows, float64 numpy"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def cpu_baseline(prob, pairs, d, Hq, heads_n):
+    from threadpoolctl import threadpool_info
+    from oracle import attention as OA
+    heads = list(range(min(heads_n, Hq)))
+    t0 = time.perf_counter()
+    OA.attention(prob.q, prob.k, prob.v, prob.mask, heads=heads)
+    sec = time.perf_counter() - t0
+    flops = 4.0 * d * pairs * len(heads) / (1 if prob.mask.Hm == 1 else Hq)
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": flops / sec / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(heads)} of {Hq} query heads, all rows, float64 numpy ({sec:.1f} s)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="doc8k", choices=sorted(BLOCKS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--oracle-heads", type=int, default=4, help="query heads in the CPU-baseline sample")
+    ap.add_argument("--reference-heads", type=int, default=1, help="query heads per reference-arm step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    prob = W.make_problem(args.workload)
+    Bsz, Hq, Hkv, N, d = prob.shape
+    pairs = visible_pairs(prob.mask)
+    flops = 4.0 * d * pairs * (Hq if prob.mask.Hm == 1 else 1)
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, prob, pairs, d, Hq)), flush=True)
+        return
+
+    import torch.distributed as dist
+    from mask_aware_block_mfa_b200 import binding as B
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    bq, bk = BLOCKS[args.workload]
+    q, k, v = (t.to(dev) for t in (prob.q, prob.k, prob.v))
+    att = B.Attention(prob.mask, bq, bk, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev_f0=None, ev_f1=None):
+        att.build(stream)
+        if ev_f0 is not None:
+            ev_f0.record(stream)
+        att(q, k, v, out, lse, stream)
+        if ev_f1 is not None:
+            ev_f1.record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize(dev)
+    if B.device_status(att.tmap, stream) != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        for e0, f0, f1, e1 in ev:
+            flush.fill_(1.0)
+            e0.record(stream)
+            step(f0, f1)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        time.sleep(0.2)
+    if world > 1:
+        dist.barrier()
+    step_ms = [e0.elapsed_time(e1) for (e0, _, _, e1) in ev]
+    fwd_ms = [f0.elapsed_time(f1) for (_, f0, f1, _) in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    fwd_avg_ms = sum(fwd_ms) / len(fwd_ms)
+    achieved = flops / (fwd_avg_ms * 1e-3) / 1e12
+    burst, sustained, src = peaks()
+
+    # End to end through the binding: pinned host inputs -> device -> map + forward -> host outputs.
+    hq, hk, hv = (t.pin_memory() for t in (prob.q, prob.k, prob.v))
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    mask_bytes = sum(getattr(prob.mask, f).nbytes for f in ("lts", "lte", "uts", "ute", "sel")
+                     if getattr(prob.mask, f) is not None)
+    h2d = hq.nbytes + hk.nbytes + hv.nbytes + mask_bytes
+    d2h = ho.nbytes + hl.nbytes
+    e2e_ms = []
+    for s in range(args.e2e_steps + 1):  # the first pass is a warm-up
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        att_e = att
+        att_e.dmask = B.DeviceMask(prob.mask, dev)  # mask arrays host -> device
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        att_e.build(stream)
+        att_e(q, k, v, out, lse, stream)
+        ho.copy_(out, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+        z.record(stream)
+        torch.cuda.synchronize(dev)
+        if s > 0:
+            e2e_ms.append(a.elapsed_time(z))
+    e2e_value = flops * world / (statistics.mean(e2e_ms) * 1e-3) / 1e12
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    res = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "desc": W.WORKLOADS[args.workload], "B": Bsz, "Hq": Hq, "Hkv": Hkv,
+                   "N": N, "d": d, "block_q": bq, "block_k": bk, "seed": prob.seed, "visible_pairs": pairs,
+                   "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}"},
+        "frac_of_peak": {"burst": value / burst, "sustained": value / sustained, "spec_2250": value / 2250.0,
+                         "peaks": src},
+        "fwd_only": {"ms": fwd_avg_ms, "tflops": achieved},
+        "map_ms": ms_per_step - fwd_avg_ms,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                     "frac": achieved / burst, "traffic": None, "peak_kind": f"{src} burst bf16 dense"},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms": statistics.mean(e2e_ms)},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        res["cpu_baseline"] = cpu_baseline(prob, pairs, d, Hq, args.oracle_heads)
+    print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,185 @@
+/*
+ * mfa.h -- mask-aware flash-attention forward pass for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libmfa.so. Two calls carry the computation:
+ *
+ *   mfa_build_tile_map  reduces a compact mask description to a per-tile
+ *                       SKIP / FULL / PARTIAL map plus, for every query tile,
+ *                       the ascending list of key tiles that must be computed
+ *                       (Binary Block Masking, "Efficiently Dispatching Flash
+ *                       Attention For Partially Filled Attention Masks",
+ *                       abstract: fully masked blocks are never processed and
+ *                       fully visible blocks need no per-element mask).
+ *   mfa_fwd             computes out = softmax(Q K^T / sqrt(d) + mask) V and the
+ *                       natural-log log-sum-exp of every query row, visiting
+ *                       only the listed key tiles (FlashMask author response:
+ *                       calculations for fully masked blocks are unnecessary).
+ *
+ * Conventions shared by every call:
+ *
+ * - All tensor and array pointers are DEVICE pointers unless a comment says
+ *   otherwise. The caller allocates and owns every buffer; the library
+ *   allocates no device memory and keeps no state between calls except a
+ *   per-process cache of kernel attributes.
+ * - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *   is the legacy default stream). Argument errors are detected on the host and
+ *   returned before anything is launched. Problems only the device can see
+ *   (bounds out of range, a bounded wait that gave up) are recorded in the tile
+ *   map's error word and reported by mfa_get_device_status.
+ * - Combinations the kernels do not implement return MFA_ERR_UNSUPPORTED; the
+ *   library never computes a silently different mask (the selected-key pull
+ *   request's lesson: a kernel must decline an op it cannot compute exactly).
+ *
+ * Mask semantics (masked = not attended):
+ * - COLWISE, FlashMask-style column-wise row intervals: for key column j, query
+ *   rows i with lts[j] <= i < lte[j] or uts[j] <= i < ute[j] are masked.
+ *   Half-open; start >= end is empty; every bound must lie in [0, Nq]. Arrays
+ *   are int32 [B, Hm, Nk], contiguous. A NULL pair (lts/lte or uts/ute) is the
+ *   empty interval. A causal mask is given explicitly as uts = 0, ute = j.
+ * - BAND, Ascend sparseMode 0 (equal to sparseMode 4 when Nq == Nk): the pair
+ *   (i, j) is attended iff -pre_tokens <= j - i <= next_tokens, both ends
+ *   inclusive (Ascend CANN "sparseMode introduction", sparseMode 0 and 4).
+ * - BLOCKSEL, per-query-block key-block lists (the selected-key flash attention
+ *   pull request): sel is int32 [B, Hm, ceil(Nq/64), sel_k]; entry -1 is no
+ *   entry, duplicates count once, entries must lie in [-1, ceil(Nk/64)).
+ *   Query i attends key j iff block j/64 is listed for block i/64 and j <= i.
+ * A query row that attends no key gets out = 0 and lse = -inf.
+ */
+#ifndef MFA_H_
+#define MFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MFA_ABI_VERSION 1
+
+typedef enum {
+  MFA_OK = 0,
+  MFA_ERR_INVALID_ARG = 1,    /* NULL pointer, negative size, bad enum value   */
+  MFA_ERR_UNSUPPORTED = 2,    /* a valid combination the kernels do not cover */
+  MFA_ERR_SHAPE_MISMATCH = 3, /* tensors, mask and map disagree on a size      */
+  MFA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed          */
+  MFA_ERR_DEVICE = 5          /* the device recorded an error (see error bits) */
+} mfa_status;
+
+typedef enum { MFA_BF16 = 0, MFA_F32 = 1 } mfa_dtype;
+
+typedef enum { MFA_MASK_COLWISE = 0, MFA_MASK_BAND = 1, MFA_MASK_BLOCKSEL = 2 } mfa_mask_kind;
+
+/* Device error word bits (mfa_tile_map.err). */
+#define MFA_DEVERR_BOUNDS 1u   /* a column bound outside [0, Nq]                      */
+#define MFA_DEVERR_SEL 2u      /* a selection entry outside [-1, ceil(Nk/64))         */
+#define MFA_DEVERR_TIMEOUT 4u  /* a bounded wait in mfa_fwd gave up; outputs invalid  */
+#define MFA_DEVERR_MAP 8u      /* mfa_fwd read a tile list entry outside [0, nkt)     */
+
+/* A 4-D tensor [B, H, N, D]; strides in ELEMENTS, stride[3] must be 1. */
+typedef struct {
+  void* data;        /* device pointer                                    */
+  int32_t dtype;     /* mfa_dtype                                         */
+  int32_t reserved;
+  int64_t B, H, N, D;
+  int64_t stride[4];
+} mfa_tensor;
+
+/* The tile map: shape fields are set by mfa_tile_map_init, the pointers carve
+ * one caller-owned device buffer of mfa_tile_map_bytes() bytes. Layout (per
+ * batch b, mask head hm; nqt = ceil(Nq/block_q), nkt = ceil(Nk/block_k)):
+ *   kminmax    int32 [B, Hm, nkt, 8]  min/max over the k-tile's columns of
+ *              LTS, LTE, UTS, UTE (in that order, min then max), with every
+ *              empty interval written as start = Nq, end = 0; the band kind is
+ *              first turned into UT = [0, clamp(j - next, 0, Nq)),
+ *              LT = [clamp(j + pre + 1, 0, Nq), Nq). Zero for BLOCKSEL.
+ *   tile_class uint8 [B, Hm, nqt, nkt] bits 0-1: 0 SKIP, 1 FULL, 2 PARTIAL.
+ *              BLOCKSEL only: bit 4 + 2*qs + ks set when 64x64 sub-block
+ *              (qs, ks) of the tile holds a visible pair.
+ *   tile_list  int32 [B, Hm, nqt, nkt] ascending non-SKIP k-tiles, -1 padded.
+ *   tile_count int32 [B, Hm, nqt].
+ *   order      int32 [B*Hm*nqt] flat (b, hm, qt) sorted by count, largest
+ *              first, ties by index (the forward pass's work order).
+ *   err        uint32 device error word (MFA_DEVERR_* bits), cleared by
+ *              mfa_build_tile_map, set by it and by mfa_fwd.
+ * Class rule for COLWISE / BAND with r0 = qt*block_q, r1 = min(r0+block_q, Nq):
+ *   SKIP    if (LTSmax <= r0 && LTEmin >= r1) || (UTSmax <= r0 && UTEmin >= r1)
+ *   FULL    else if (LTSmin >= r1 || LTEmax <= r0) && (UTSmin >= r1 || UTEmax <= r0)
+ *   PARTIAL otherwise.
+ * BLOCKSEL: SKIP if every valid 64x64 sub-block is unlisted or above the
+ * diagonal block, FULL if every one is listed and strictly below it. */
+typedef struct mfa_tile_map {
+  int32_t B, Hm, Nq, Nk, block_q, block_k, nqt, nkt;
+  int32_t kind;      /* mask kind of the last mfa_build_tile_map (-1 before) */
+  int32_t reserved;
+  int32_t* kminmax;
+  uint8_t* tile_class;
+  int32_t* tile_list;
+  int32_t* tile_count;
+  int32_t* order;
+  uint32_t* err;
+} mfa_tile_map;
+
+/* A compact mask description. Sizes: B batch, Hm mask heads (1 = one mask
+ * shared by all query heads, or Hq = one per query head), Nq queries, Nk keys. */
+typedef struct {
+  int32_t kind;                   /* mfa_mask_kind                            */
+  int32_t B, Hm, Nq, Nk;
+  int32_t sel_k;                  /* BLOCKSEL: entries per query block        */
+  int32_t sel_block;              /* BLOCKSEL: must be 64                     */
+  int32_t reserved;
+  const int32_t *lts, *lte, *uts, *ute; /* COLWISE: device int32 [B, Hm, Nk]  */
+  int64_t pre_tokens, next_tokens;      /* BAND                               */
+  const int32_t* sel;                   /* BLOCKSEL: device int32 [B,Hm,nqb,sel_k] */
+  const mfa_tile_map* map;              /* mfa_fwd: the map built from this mask */
+} mfa_mask_desc;
+
+/* ABI version of the loaded library (MFA_ABI_VERSION). Host only. */
+int32_t mfa_abi_version(void);
+
+/* Human-readable name of a status code. Host only; never NULL. */
+const char* mfa_status_string(mfa_status s);
+
+/* Bytes of device memory a tile map of this shape needs (0 on bad arguments).
+ * block_q and block_k must each be 64 or 128. Host only. */
+size_t mfa_tile_map_bytes(int32_t B, int32_t Hm, int32_t Nq, int32_t Nk,
+                          int32_t block_q, int32_t block_k);
+
+/* Fill `map` (host struct) with the shape and with pointers into `device_buf`
+ * (caller-owned, 256-byte aligned, at least mfa_tile_map_bytes() bytes). No
+ * device work. Returns INVALID_ARG / UNSUPPORTED on bad arguments. */
+mfa_status mfa_tile_map_init(mfa_tile_map* map, void* device_buf, size_t bytes,
+                             int32_t B, int32_t Hm, int32_t Nq, int32_t Nk,
+                             int32_t block_q, int32_t block_k);
+
+/* Build `map` from `mask` on `stream`: clears err, computes kminmax,
+ * tile_class, tile_list, tile_count and order (three kernel launches). The
+ * mask's shape must equal the map's. mask->map is ignored. Device-detected
+ * range errors set MFA_DEVERR_BOUNDS / MFA_DEVERR_SEL. */
+mfa_status mfa_build_tile_map(const mfa_mask_desc* mask, mfa_tile_map* map, void* stream);
+
+/* Attention forward pass on `stream`.
+ *   q   [B, Hq, Nq, D], k and v [B, Hkv, Nk, D], out [B, Hq, Nq, D]: dtype
+ *       MFA_BF16 (MFA_F32 is rejected as UNSUPPORTED), D in {64, 128},
+ *       Hq % Hkv == 0 (query head h reads key/value head h / (Hq/Hkv)),
+ *       stride[3] == 1, other strides and the base address 16-byte aligned.
+ *   mask  description with mask->map built from it by mfa_build_tile_map
+ *         (same kind and shape); Hm must be 1 or Hq.
+ *   lse   float32 [B, Hq, Nq] contiguous, natural-log log-sum-exp per row.
+ * Query tiles pack heads: block_q == 128 puts 128 queries of one head in a
+ * tile; block_q == 64 puts 64 queries of two heads of one key/value group in
+ * a tile and needs Hm == 1 and an even Hq/Hkv. block_k is 64 or 128.
+ * Rows with no visible key get out = 0 and lse = -inf. */
+mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v,
+                   const mfa_mask_desc* mask, const mfa_tensor* out, float* lse,
+                   void* stream);
+
+/* Synchronise `stream`, read the map's error word into *err_bits (if not
+ * NULL) and return MFA_ERR_DEVICE when it is non-zero, MFA_OK otherwise. */
+mfa_status mfa_get_device_status(const mfa_tile_map* map, void* stream, uint32_t* err_bits);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MFA_H_ */

@@ -1,0 +1,221 @@
+"""Thin ctypes binding of libmfa.so (argument marshalling only).
+
+Every computation runs in the library's CUDA kernels; this module only turns
+torch tensors and mask descriptions into the C structs of ``include/mfa.h``
+and calls the entry points of the same names. It raises if the library is
+missing or a call fails: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import workloads as W
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmfa.so")
+
+MFA_OK, MFA_ERR_INVALID_ARG, MFA_ERR_UNSUPPORTED, MFA_ERR_SHAPE_MISMATCH, MFA_ERR_CUDA, MFA_ERR_DEVICE = range(6)
+MFA_BF16, MFA_F32 = 0, 1
+DEVERR_BOUNDS, DEVERR_SEL, DEVERR_TIMEOUT, DEVERR_MAP = 1, 2, 4, 8
+
+EXPORTS = ("mfa_abi_version", "mfa_status_string", "mfa_tile_map_bytes", "mfa_tile_map_init",
+           "mfa_build_tile_map", "mfa_fwd", "mfa_get_device_status")
+
+
+class MfaTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("B", ctypes.c_int64), ("H", ctypes.c_int64), ("N", ctypes.c_int64), ("D", ctypes.c_int64),
+                ("stride", ctypes.c_int64 * 4)]
+
+
+class MfaTileMap(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hm", ctypes.c_int32), ("Nq", ctypes.c_int32), ("Nk", ctypes.c_int32),
+                ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32), ("nqt", ctypes.c_int32),
+                ("nkt", ctypes.c_int32), ("kind", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("kminmax", ctypes.c_void_p), ("tile_class", ctypes.c_void_p), ("tile_list", ctypes.c_void_p),
+                ("tile_count", ctypes.c_void_p), ("order", ctypes.c_void_p), ("err", ctypes.c_void_p)]
+
+
+class MfaMaskDesc(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("B", ctypes.c_int32), ("Hm", ctypes.c_int32), ("Nq", ctypes.c_int32),
+                ("Nk", ctypes.c_int32), ("sel_k", ctypes.c_int32), ("sel_block", ctypes.c_int32),
+                ("reserved", ctypes.c_int32),
+                ("lts", ctypes.c_void_p), ("lte", ctypes.c_void_p), ("uts", ctypes.c_void_p), ("ute", ctypes.c_void_p),
+                ("pre_tokens", ctypes.c_int64), ("next_tokens", ctypes.c_int64),
+                ("sel", ctypes.c_void_p), ("map", ctypes.POINTER(MfaTileMap))]
+
+
+class MfaError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} returned {status} ({msg})")
+        self.status = status
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load(path: str = _LIB_PATH) -> ctypes.CDLL:
+    """Load libmfa.so (built in-tree by mask_aware_block_mfa_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: run `python -m mask_aware_block_mfa_b200.build`")
+    lib = ctypes.CDLL(path)
+    lib.mfa_abi_version.restype = ctypes.c_int32
+    lib.mfa_status_string.restype = ctypes.c_char_p
+    lib.mfa_status_string.argtypes = [ctypes.c_int]
+    lib.mfa_tile_map_bytes.restype = ctypes.c_size_t
+    lib.mfa_tile_map_bytes.argtypes = [ctypes.c_int32] * 6
+    lib.mfa_tile_map_init.restype = ctypes.c_int
+    lib.mfa_tile_map_init.argtypes = [ctypes.POINTER(MfaTileMap), ctypes.c_void_p, ctypes.c_size_t] + [ctypes.c_int32] * 6
+    lib.mfa_build_tile_map.restype = ctypes.c_int
+    lib.mfa_build_tile_map.argtypes = [ctypes.POINTER(MfaMaskDesc), ctypes.POINTER(MfaTileMap), ctypes.c_void_p]
+    lib.mfa_fwd.restype = ctypes.c_int
+    lib.mfa_fwd.argtypes = [ctypes.POINTER(MfaTensor)] * 3 + [ctypes.POINTER(MfaMaskDesc), ctypes.POINTER(MfaTensor),
+                                                              ctypes.c_void_p, ctypes.c_void_p]
+    lib.mfa_get_device_status.restype = ctypes.c_int
+    lib.mfa_get_device_status.argtypes = [ctypes.POINTER(MfaTileMap), ctypes.c_void_p,
+                                          ctypes.POINTER(ctypes.c_uint32)]
+    if lib.mfa_abi_version() != 1:
+        raise RuntimeError("libmfa.so ABI version mismatch")
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().mfa_status_string(code).decode()
+
+
+def _check(fn: str, code: int) -> None:
+    if code != MFA_OK:
+        raise MfaError(fn, code, status_string(code))
+
+
+def tensor_desc(t: torch.Tensor) -> MfaTensor:
+    if t.dim() != 4:
+        raise ValueError("expected a [B, H, N, D] tensor")
+    dt = {torch.bfloat16: MFA_BF16, torch.float32: MFA_F32}.get(t.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    d = MfaTensor()
+    d.data = t.data_ptr()
+    d.dtype = dt
+    d.B, d.H, d.N, d.D = (int(x) for x in t.shape)
+    for i in range(4):
+        d.stride[i] = int(t.stride(i))
+    return d
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+class DeviceMask:
+    """A mask description whose arrays live on the device, plus its C struct."""
+
+    def __init__(self, mask: W.MaskDesc, device="cuda"):
+        self.mask = mask
+        self._keep = []
+        d = MfaMaskDesc()
+        d.kind, d.B, d.Hm, d.Nq, d.Nk = mask.kind, mask.B, mask.Hm, mask.Nq, mask.Nk
+        d.sel_k, d.sel_block = mask.sel_k, mask.sel_block
+        for f in ("lts", "lte", "uts", "ute", "sel"):
+            a = getattr(mask, f)
+            if a is None:
+                setattr(d, f, None)
+                continue
+            t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+            self._keep.append(t)
+            setattr(d, f, t.data_ptr())
+        d.pre_tokens, d.next_tokens = int(mask.pre_tokens), int(mask.next_tokens)
+        d.map = None
+        self.desc = d
+
+
+class TileMap:
+    """A tile map in one caller-owned device buffer (see mfa_tile_map in mfa.h)."""
+
+    def __init__(self, B, Hm, Nq, Nk, block_q, block_k, device="cuda"):
+        lib = load()
+        nbytes = lib.mfa_tile_map_bytes(B, Hm, Nq, Nk, block_q, block_k)
+        if nbytes == 0:
+            raise MfaError("mfa_tile_map_bytes", MFA_ERR_INVALID_ARG, "bad shape or block sizes")
+        self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        base = self.buf.data_ptr()
+        aligned = (base + 255) & ~255
+        self.m = MfaTileMap()
+        _check("mfa_tile_map_init", lib.mfa_tile_map_init(ctypes.byref(self.m), aligned, nbytes,
+                                                          B, Hm, Nq, Nk, block_q, block_k))
+        self.offset = aligned - base
+        self.nbytes = nbytes
+
+    def arrays(self):
+        """Views of the map arrays as torch tensors on the device."""
+        m = self.m
+        BH, nqt, nkt = m.B * m.Hm, m.nqt, m.nkt
+
+        def view(ptr, dtype, count):
+            off = ptr - self.buf.data_ptr()
+            el = torch.tensor([], dtype=dtype).element_size()
+            return self.buf[off:off + count * el].view(dtype)
+
+        return {
+            "kminmax": view(m.kminmax, torch.int32, BH * nkt * 8).view(m.B, m.Hm, nkt, 8),
+            "tile_class": view(m.tile_class, torch.uint8, BH * nqt * nkt).view(m.B, m.Hm, nqt, nkt),
+            "tile_list": view(m.tile_list, torch.int32, BH * nqt * nkt).view(m.B, m.Hm, nqt, nkt),
+            "tile_count": view(m.tile_count, torch.int32, BH * nqt).view(m.B, m.Hm, nqt),
+            "order": view(m.order, torch.int32, BH * nqt),
+            "err": view(m.err, torch.int32, 1),
+        }
+
+
+def build_tile_map(dmask: DeviceMask, tmap: TileMap, stream=None) -> None:
+    _check("mfa_build_tile_map", load().mfa_build_tile_map(ctypes.byref(dmask.desc), ctypes.byref(tmap.m),
+                                                           _stream_ptr(stream)))
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: DeviceMask, tmap: TileMap,
+        out: torch.Tensor, lse: torch.Tensor, stream=None) -> None:
+    """out, lse <- attention(q, k, v) under dmask, through the tile map (both on the device)."""
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor")
+    dmask.desc.map = ctypes.pointer(tmap.m)
+    qd, kd, vd, od = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
+    _check("mfa_fwd", load().mfa_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(dmask.desc),
+                                     ctypes.byref(od), lse.data_ptr(), _stream_ptr(stream)))
+
+
+def device_status(tmap: TileMap, stream=None) -> int:
+    """Synchronise and return the map's device error bits (0 = none)."""
+    bits = ctypes.c_uint32(0)
+    code = load().mfa_get_device_status(ctypes.byref(tmap.m), _stream_ptr(stream), ctypes.byref(bits))
+    if code not in (MFA_OK, MFA_ERR_DEVICE):
+        _check("mfa_get_device_status", code)
+    return int(bits.value)
+
+
+class Attention:
+    """Convenience wrapper: upload a mask, build its map once, run forward passes."""
+
+    def __init__(self, mask: W.MaskDesc, block_q: int = 64, block_k: int = 128, device="cuda"):
+        self.dmask = DeviceMask(mask, device)
+        self.tmap = TileMap(mask.B, mask.Hm, mask.Nq, mask.Nk, block_q, block_k, device)
+        self.device = device
+
+    def build(self, stream=None):
+        build_tile_map(self.dmask, self.tmap, stream)
+
+    def __call__(self, q, k, v, out=None, lse=None, stream=None):
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        fwd(q, k, v, self.dmask, self.tmap, out, lse, stream)
+        return out, lse

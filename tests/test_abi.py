@@ -1,0 +1,185 @@
+"""The C ABI on the host: exports, struct layouts and argument validation.
+
+Nothing here touches a GPU: every call below is rejected by host-side checks
+before the library makes a CUDA call, or only carves pointers.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from mask_aware_block_mfa_b200 import binding as B
+from mask_aware_block_mfa_b200 import build as BUILD
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mfa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    BUILD.build()
+    return B.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mfa_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_function_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(B.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", BUILD.LIB], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (mfa_\w+)", out))
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+
+
+def test_struct_layouts_match_header(tmp_path):
+    src = tmp_path / "layout.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <stddef.h>
+#include "mfa.h"
+#define F(T, f) printf(#T "." #f " %zu\n", offsetof(T, f))
+int main(void) {
+  printf("mfa_tensor %zu\nmfa_tile_map %zu\nmfa_mask_desc %zu\n",
+         sizeof(mfa_tensor), sizeof(mfa_tile_map), sizeof(mfa_mask_desc));
+  F(mfa_tensor, data); F(mfa_tensor, B); F(mfa_tensor, stride);
+  F(mfa_tile_map, kind); F(mfa_tile_map, kminmax); F(mfa_tile_map, err);
+  F(mfa_mask_desc, lts); F(mfa_mask_desc, pre_tokens); F(mfa_mask_desc, sel); F(mfa_mask_desc, map);
+  return 0;
+}''')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True).stdout.splitlines())
+    assert int(got["mfa_tensor"]) == ctypes.sizeof(B.MfaTensor)
+    assert int(got["mfa_tile_map"]) == ctypes.sizeof(B.MfaTileMap)
+    assert int(got["mfa_mask_desc"]) == ctypes.sizeof(B.MfaMaskDesc)
+    for key, val in got.items():
+        if "." in key:
+            struct, field = key.split(".")
+            cls = {"mfa_tensor": B.MfaTensor, "mfa_tile_map": B.MfaTileMap, "mfa_mask_desc": B.MfaMaskDesc}[struct]
+            assert getattr(cls, field).offset == int(val), key
+
+
+def test_status_strings(lib):
+    assert lib.mfa_abi_version() == 1
+    for code in range(6):
+        assert lib.mfa_status_string(code)
+    assert lib.mfa_status_string(99) == b"unknown status"
+
+
+def test_tile_map_bytes_and_init(lib):
+    assert lib.mfa_tile_map_bytes(1, 1, 8192, 8192, 64, 128) > 0
+    assert lib.mfa_tile_map_bytes(1, 1, 8192, 8192, 32, 128) == 0
+    assert lib.mfa_tile_map_bytes(0, 1, 8192, 8192, 64, 128) == 0
+    nb = lib.mfa_tile_map_bytes(2, 1, 1000, 900, 64, 64)
+    nqt, nkt = 16, 15
+    expect = 0
+    for sz in (2 * nkt * 8 * 4, 2 * nqt * nkt, 2 * nqt * nkt * 4, 2 * nqt * 4, 2 * nqt * 4, 4):
+        expect += (sz + 255) // 256 * 256
+    assert nb == expect
+    m = B.MfaTileMap()
+    fake = 0x7000_0000_0000
+    assert lib.mfa_tile_map_init(ctypes.byref(m), fake, nb, 2, 1, 1000, 900, 64, 64) == B.MFA_OK
+    assert (m.nqt, m.nkt, m.kind) == (nqt, nkt, -1)
+    assert m.kminmax == fake and m.err > m.order > m.tile_count > m.tile_list > m.tile_class > m.kminmax
+    assert all(p % 256 == 0 for p in (m.kminmax, m.tile_class, m.tile_list, m.tile_count, m.order, m.err))
+    assert lib.mfa_tile_map_init(ctypes.byref(m), fake, nb - 1, 2, 1, 1000, 900, 64, 64) == B.MFA_ERR_INVALID_ARG
+    assert lib.mfa_tile_map_init(ctypes.byref(m), fake + 16, nb, 2, 1, 1000, 900, 64, 64) == B.MFA_ERR_INVALID_ARG
+    assert lib.mfa_tile_map_init(ctypes.byref(m), None, nb, 2, 1, 1000, 900, 64, 64) == B.MFA_ERR_INVALID_ARG
+    assert lib.mfa_tile_map_init(ctypes.byref(m), fake, nb, 2, 1, 1000, 900, 96, 64) == B.MFA_ERR_UNSUPPORTED
+
+
+def _fake_map(lib, Bsz=1, Hm=1, Nq=512, Nk=512, bq=64, bk=128, kind=0):
+    m = B.MfaTileMap()
+    nb = lib.mfa_tile_map_bytes(Bsz, Hm, Nq, Nk, bq, bk)
+    assert lib.mfa_tile_map_init(ctypes.byref(m), 0x7000_0000_0000, nb, Bsz, Hm, Nq, Nk, bq, bk) == 0
+    m.kind = kind
+    return m
+
+
+def _fake_tensor(Bsz, H, N, D, dtype=B.MFA_BF16, addr=0x7100_0000_0000):
+    t = B.MfaTensor()
+    t.data, t.dtype = addr, dtype
+    t.B, t.H, t.N, t.D = Bsz, H, N, D
+    t.stride[0], t.stride[1], t.stride[2], t.stride[3] = H * N * D, N * D, D, 1
+    return t
+
+
+def _fake_mask(m, kind=0, Bsz=1, Hm=1, Nq=512, Nk=512):
+    d = B.MfaMaskDesc()
+    d.kind, d.B, d.Hm, d.Nq, d.Nk = kind, Bsz, Hm, Nq, Nk
+    d.sel_block = 64
+    d.map = ctypes.pointer(m)
+    return d
+
+
+def _fwd(lib, q, k, v, d, o, lse=0x7200_0000_0000):
+    return lib.mfa_fwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.byref(d), ctypes.byref(o),
+                       lse, None)
+
+
+def test_fwd_rejects_bad_arguments_on_host(lib):
+    m = _fake_map(lib)
+    q, k, v, o = _fake_tensor(1, 8, 512, 128), _fake_tensor(1, 2, 512, 128), _fake_tensor(1, 2, 512, 128), \
+        _fake_tensor(1, 8, 512, 128)
+    d = _fake_mask(m)
+    assert _fwd(lib, q, k, v, d, o, lse=0) == B.MFA_ERR_INVALID_ARG
+    qn = _fake_tensor(1, 8, 512, 128, addr=0)
+    assert _fwd(lib, qn, k, v, d, o) == B.MFA_ERR_INVALID_ARG
+    q32 = _fake_tensor(1, 8, 512, 128, dtype=B.MFA_F32)
+    o32 = _fake_tensor(1, 8, 512, 128, dtype=B.MFA_F32)
+    k32, v32 = _fake_tensor(1, 2, 512, 128, dtype=B.MFA_F32), _fake_tensor(1, 2, 512, 128, dtype=B.MFA_F32)
+    assert _fwd(lib, q32, k32, v32, d, o32) == B.MFA_ERR_UNSUPPORTED          # fp32 not implemented
+    assert _fwd(lib, q32, k, v, d, o) == B.MFA_ERR_INVALID_ARG                # mixed dtypes
+    assert _fwd(lib, _fake_tensor(1, 8, 512, 96), _fake_tensor(1, 2, 512, 96), _fake_tensor(1, 2, 512, 96), d,
+                _fake_tensor(1, 8, 512, 96)) == B.MFA_ERR_UNSUPPORTED         # head dim 96
+    assert _fwd(lib, q, _fake_tensor(1, 3, 512, 128), _fake_tensor(1, 3, 512, 128), d, o) == \
+        B.MFA_ERR_SHAPE_MISMATCH                                              # Hq % Hkv != 0
+    assert _fwd(lib, q, k, _fake_tensor(1, 2, 256, 128), d, o) == B.MFA_ERR_SHAPE_MISMATCH
+    assert _fwd(lib, q, k, v, d, _fake_tensor(1, 8, 256, 128)) == B.MFA_ERR_SHAPE_MISMATCH
+    bad_stride = _fake_tensor(1, 8, 512, 128)
+    bad_stride.stride[3] = 2
+    assert _fwd(lib, bad_stride, k, v, d, o) == B.MFA_ERR_UNSUPPORTED
+    unaligned = _fake_tensor(1, 8, 512, 128, addr=0x7100_0000_0002)
+    assert _fwd(lib, unaligned, k, v, d, o) == B.MFA_ERR_UNSUPPORTED
+    # mask / map disagreements
+    d2 = _fake_mask(m, Nq=256)
+    assert _fwd(lib, q, k, v, d2, o) == B.MFA_ERR_SHAPE_MISMATCH
+    d3 = _fake_mask(m, kind=1)                                                # map built from another kind
+    assert _fwd(lib, q, k, v, d3, o) == B.MFA_ERR_SHAPE_MISMATCH
+    d4 = _fake_mask(m)
+    d4.map = None
+    assert _fwd(lib, q, k, v, d4, o) == B.MFA_ERR_INVALID_ARG
+    # two heads per tile (block_q = 64) need an even group size and one mask head
+    q6 = _fake_tensor(1, 6, 512, 128)
+    k6, v6 = _fake_tensor(1, 2, 512, 128), _fake_tensor(1, 2, 512, 128)
+    assert _fwd(lib, q6, k6, v6, d, _fake_tensor(1, 6, 512, 128)) == B.MFA_ERR_UNSUPPORTED
+    m8 = _fake_map(lib, Hm=8)
+    d8 = _fake_mask(m8, Hm=8)
+    assert _fwd(lib, q, k, v, d8, o) == B.MFA_ERR_UNSUPPORTED
+    m3 = _fake_map(lib, Hm=3, bq=128)
+    assert _fwd(lib, q, k, v, _fake_mask(m3, Hm=3), o) == B.MFA_ERR_SHAPE_MISMATCH  # Hm not in {1, Hq}
+
+
+def test_build_rejects_bad_arguments_on_host(lib):
+    m = _fake_map(lib)
+    d = _fake_mask(m)
+    assert lib.mfa_build_tile_map(None, ctypes.byref(m), None) == B.MFA_ERR_INVALID_ARG
+    assert lib.mfa_build_tile_map(ctypes.byref(d), None, None) == B.MFA_ERR_INVALID_ARG
+    bad = _fake_mask(m, kind=7)
+    assert lib.mfa_build_tile_map(ctypes.byref(bad), ctypes.byref(m), None) == B.MFA_ERR_INVALID_ARG
+    other = _fake_mask(m, Nk=256)
+    assert lib.mfa_build_tile_map(ctypes.byref(other), ctypes.byref(m), None) == B.MFA_ERR_SHAPE_MISMATCH
+    sel = _fake_mask(m, kind=2)
+    assert lib.mfa_build_tile_map(ctypes.byref(sel), ctypes.byref(m), None) == B.MFA_ERR_INVALID_ARG  # no list
+    sel.sel, sel.sel_k, sel.sel_block = 0x7300_0000_0000, 16, 32
+    assert lib.mfa_build_tile_map(ctypes.byref(sel), ctypes.byref(m), None) == B.MFA_ERR_UNSUPPORTED
+    m.tile_list = None
+    assert lib.mfa_build_tile_map(ctypes.byref(d), ctypes.byref(m), None) == B.MFA_ERR_INVALID_ARG

@@ -1,0 +1,126 @@
+"""GPU forward pass vs the float64 oracle, element by element.
+
+Small problems are compared on every row (they span several tiles and end in
+ragged tails); the named full-size workloads, in the launch configuration the
+benchmark times, are compared on sampled rows of sampled heads.
+Tolerances: max |out - ref| <= 2e-2, mean <= 2e-3, |lse - ref| <= 1e-3 on rows
+with a visible key; rows without one must give exactly out = 0, lse = -inf.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from mask_aware_block_mfa_b200 import binding as B
+from mask_aware_block_mfa_b200 import workloads as W
+
+from .gpu_util import compare_attention, compare_map, oracle_rows, run_gpu, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def small_problem(mask, Hq, Hkv, d, seed, Nq=None, Nk=None):
+    Nq = mask.Nq if Nq is None else Nq
+    Nk = mask.Nk if Nk is None else Nk
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(mask.B, Hq, Nq, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(mask.B, Hkv, Nk, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(mask.B, Hkv, Nk, d, generator=g).to(torch.bfloat16)
+    return W.Problem("small", q, k, v, mask, seed)
+
+
+def check_full(prob, bq, bk):
+    out, lse, arrays, err = run_gpu(prob, bq, bk)
+    assert err == 0
+    compare_map(arrays, prob.mask, bq, bk)
+    ref_out, ref_lse = oracle_rows(prob, None)
+    return compare_attention(out, lse, ref_out, ref_lse)
+
+
+RNG = np.random.default_rng(5)
+CASES = [
+    # name, mask, Hq, Hkv, d, block sizes
+    ("doc_gqa", W.make_mask("doc8k", N=1024), 8, 2, 128, [(64, 128), (128, 128), (64, 64), (128, 64)]),
+    ("doc_ragged", W.make_mask("tiny_doc_fp32", N=1000), 4, 2, 128, [(64, 128), (128, 64)]),
+    ("shared", W.make_mask("shared_question8k", N=2048), 4, 2, 128, [(64, 128)]),
+    ("band", W.band(2, 1500, 300, 0), 2, 2, 128, [(128, 128), (128, 64)]),
+    ("band_neg", W.band(1, 900, 400, -64), 2, 2, 128, [(128, 128)]),
+    ("band_negpre", W.band(1, 700, -40, 170), 2, 1, 128, [(128, 128), (64, 64)]),
+    ("blocksel", W.blocksel_topk(RNG, 1, 1024, 4), 4, 2, 128, [(64, 64), (64, 128), (128, 128)]),
+    ("blocksel_rand", W.random_blocksel(RNG, 1, 700, 700, 5), 2, 1, 128, [(64, 64), (128, 128)]),
+    ("random_hm", W.random_colwise(RNG, 1, 4, 700, 700), 4, 2, 128, [(128, 128), (128, 64)]),
+    ("doc_d64", W.make_mask("doc8k", N=1024), 4, 2, 64, [(64, 128), (128, 64)]),
+    ("band_d64", W.band(1, 777, 100, 3), 2, 2, 64, [(128, 128)]),
+]
+
+
+@pytest.mark.parametrize("name,mask,Hq,Hkv,d,blocks", CASES, ids=[c[0] for c in CASES])
+def test_fwd_small_all_rows(name, mask, Hq, Hkv, d, blocks):
+    prob = small_problem(mask, Hq, Hkv, d, seed=zlib.crc32(name.encode()) % 1000)
+    for bq, bk in blocks:
+        check_full(prob, bq, bk)
+
+
+def test_fwd_rectangular_nq_ne_nk():
+    rng = np.random.default_rng(9)
+    mask = W.random_colwise(rng, 1, 1, 500, 900)
+    prob = small_problem(mask, 4, 2, 128, seed=3, Nq=500, Nk=900)
+    check_full(prob, 64, 128)
+
+
+def test_fwd_no_keys():
+    """Nk = 0: every row sees nothing."""
+    mask = W.MaskDesc(W.MASK_COLWISE, 1, 1, 200, 0)
+    prob = small_problem(mask, 4, 2, 128, seed=2, Nq=200, Nk=0)
+    out, lse, _, err = run_gpu(prob, 64, 128)
+    assert err == 0
+    assert torch.isneginf(lse).all() and (out == 0).all()
+
+
+def test_fwd_all_rows_masked():
+    prob = small_problem(W.band(1, 300, 10, -400), 2, 2, 128, seed=4)
+    out, lse, _, err = run_gpu(prob, 128, 128)
+    assert err == 0
+    assert torch.isneginf(lse).all() and (out == 0).all()
+
+
+def test_fwd_deterministic():
+    prob = small_problem(W.make_mask("doc8k", N=1024), 4, 2, 128, seed=6)
+    a, la, _, _ = run_gpu(prob, 64, 128)
+    b, lb, _, _ = run_gpu(prob, 64, 128)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+def test_fwd_zero_query_closed_form():
+    """q = 0 makes every visible score 0: out is the mean of the visible v rows."""
+    mask = W.make_mask("shared_question8k", N=1024)
+    prob = small_problem(mask, 2, 1, 128, seed=8)
+    prob.q.zero_()
+    out, lse, _, err = run_gpu(prob, 64, 128)
+    assert err == 0
+    ref_out, ref_lse = oracle_rows(prob, None)
+    compare_attention(out, lse, ref_out, ref_lse)
+
+
+# Full-size named workloads in the benchmark's launch configuration.
+FULL = [("doc8k", 64, 128), ("shared_question8k", 64, 128), ("band16k", 128, 128), ("band16k_neg", 128, 128),
+        ("doc32k", 64, 128), ("blocksel32k", 64, 64)]
+
+
+@pytest.mark.parametrize("name,bq,bk", FULL, ids=[f[0] for f in FULL])
+def test_fwd_full_size_sampled(name, bq, bk):
+    prob = W.make_problem(name)
+    out, lse, arrays, err = run_gpu(prob, bq, bk)
+    assert err == 0
+    compare_map(arrays, prob.mask, bq, bk)
+    rng = np.random.default_rng(17)
+    Bsz, Hq, _, N, _ = prob.shape
+    rows = sample_rows(N, 96, rng)
+    heads = sorted(set([0, Hq - 1] + [int(x) for x in rng.choice(Hq, 2, replace=False)]))
+    ref_out, ref_lse = oracle_rows(prob, rows, heads)
+    got_out = out[:, heads][:, :, rows]
+    got_lse = lse[:, heads][:, :, rows]
+    compare_attention(got_out, got_lse, ref_out, ref_lse)
+    if name == "band16k_neg":   # 64 rows per (b, h) see no key
+        assert torch.isneginf(lse[:, :, :64]).all() and torch.isfinite(lse[:, :, 64:]).all()
