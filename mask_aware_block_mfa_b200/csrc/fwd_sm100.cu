@@ -7,19 +7,34 @@
 // the exact element mask of the compact description (FlashMask's column-wise
 // intervals, the Ascend band, or 64-block selection lists).
 //
-// One CTA computes one 128-row query tile (128 queries of one head, or 64
-// queries of two heads of one key/value group when the map is built at
-// block_q = 64). Warp roles:
-//   warp 0     TMA producer: Q tile once, then K and V tiles of the listed
-//              k-tiles into two-stage shared-memory rings.
-//   warp 1     TMEM owner and MMA issuer: S = Q K^T into one of two TMEM S
-//              buffers, then O += P V with P read from TMEM.
-//   warps 4-7  softmax: one query row per thread (TMEM lane = row). Load S,
-//              mask (PARTIAL tiles only), online max / exp2 / sum, rescale O
-//              in TMEM when the running max grows, write P as bf16 over S,
-//              and finally normalise O and store out and lse.
+// Persistent kernel, one CTA per SM. A work item is two 128-row query tiles
+// that read the same key/value head:
+//   kind 0  two head tiles of one key/value group at the same query block;
+//           the mask is shared by all heads, so both tiles have the same list.
+//   kind 1  two consecutive query tiles of one head tile (used when a group
+//           holds an odd number of head tiles, or the mask has one head per
+//           query head); the MMA warp walks the union of the two lists.
+// A query tile is 128 queries of one head (block_q = 128) or 64 queries of two
+// heads of one group (block_q = 64).
+//
+// Warp roles (384 threads, three warpgroups):
+//   WG0 warp 0   TMA producer: Q of each tile once per item, then K and V of
+//                every k-tile of the union list into shared-memory rings.
+//   WG0 warp 1   TMEM owner and MMA issuer. Per k-tile and tile t: first the
+//                pending O_t += P_t V of the previous k-tile (P_t read from
+//                TMEM), then S_t = Q_t K^T. The two tiles alternate, so while
+//                one softmax warpgroup works the tensor core runs the other
+//                tile's MMAs.
+//   WG1, WG2     softmax + epilogue of tile slot 0 and 1: one row per thread
+//                (TMEM lane = row); load S, mask only PARTIAL tiles, online
+//                max / exp2 / sum, rescale O in TMEM when the running max
+//                grows by more than 2^8, write P (bf16) over S; at the end of
+//                an item read O, release it to the next item, normalise and
+//                store out and lse.
+// TMEM columns: S0 [0, BK), S1 [BK, 2BK), O0 [2BK, 2BK+D), O1 [2BK+D, 2BK+2D).
 // Every mbarrier wait is bounded; a wait that gives up raises an abort flag
 // for the whole CTA and sets MFA_DEVERR_TIMEOUT in the map's error word.
+#include <climits>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -34,14 +49,18 @@
 namespace mfa {
 namespace {
 
-constexpr int kRows = 128;       // MMA M: query rows per tile
-constexpr int kStagesK = 2;
-constexpr int kStagesV = 2;
-constexpr int kThreads = 256;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only when the max grows by > 2^8
+constexpr int kRows = 128;  // MMA M: query rows per tile
+constexpr int kThreads = 384;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 =
+// 64512); WG0 drops to 56 and the two softmax warpgroups rise to 224:
+// 128 x 56 + 256 x 224 = 64512.
+constexpr int kRegsLow = 56;
+constexpr int kRegsHigh = 224;
 
 struct FwdParams {
-  int32_t B, Hq, Hkv, G, Hm, Nq, Nk, nqt, nkt, hpe;
+  int32_t B, Hq, Hkv, G, Hm, Nq, Nk, nqt, nkt;
+  int32_t item_kind, n_items, pairs, n_ht, nqp;
   float scale_log2;  // log2(e) / sqrt(d)
   MaskArgs mask;
   const uint8_t* cls;
@@ -55,23 +74,111 @@ struct FwdParams {
 };
 
 template <int D, int BK>
-struct Smem {
-  static constexpr int kChunks = D / 64;                 // 128-byte K chunks per row
+struct Cfg {
+  static constexpr int kStages = BK == 128 ? 2 : 4;
+  static constexpr int kChunks = D / 64;  // 128-byte K chunks per row
   static constexpr int kQBytes = kRows * D * 2;
   static constexpr int kKVBytes = BK * D * 2;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kQBytes;
-  static constexpr int kV = kK + kStagesK * kKVBytes;
-  static constexpr int kBar = kV + kStagesV * kKVBytes;
-  // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], o_done,
-  // drain, bnd_full[2]
-  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 1 + 1 + 2;
-  static constexpr int kBounds = kBar + ((kNumBars * 8 + 15) / 16) * 16;  // int4 [2][BK]
-  static constexpr int kMisc = kBounds + 2 * BK * 16;
+  static constexpr int kQ = 0;  // two Q slots
+  static constexpr int kK = kQ + 2 * kQBytes;
+  static constexpr int kV = kK + kStages * kKVBytes;
+  static constexpr int kBar = kV + kStages * kKVBytes;
+  // q_full[2] q_empty[2] k_full[S] k_empty[S] v_full[S] v_empty[S] s_full[2] p_full[2]
+  // o_done[2] bnd[2][2] drain
+  static constexpr int kNumBars = 4 + 4 * kStages + 6 + 4 + 1;
+  static constexpr int kBounds = kBar + ((kNumBars * 8 + 15) / 16) * 16;  // int4 [2 tiles][2 slots][BK]
+  static constexpr int kMisc = kBounds + 4 * BK * 16;
   static constexpr int kBytes = kMisc + 16;
-  static constexpr int kAlloc = kBytes + 1024;           // slack for 1024-byte alignment
-  static constexpr int kTmemCols = (2 * BK + D) <= 256 ? 256 : 512;
+  static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+  static constexpr int kTmemCols = (2 * BK + 2 * D) <= 256 ? 256 : 512;
 };
+
+struct Tile {
+  int n;         // listed k-tiles (0: no visible key in the tile)
+  int h0, q0;    // first head and first query of the tile
+  int b;
+  bool valid;    // false when a kind-1 item runs past the last query tile
+  size_t bh_mask;
+  const int32_t* lst;
+  const uint8_t* cls;
+};
+
+template <int GP>
+__device__ __forceinline__ void decode_item(const FwdParams& p, int w, Tile (&t)[2], int& hkv) {
+  constexpr int BQ = kRows / GP;
+  if (p.item_kind == 0) {
+    const int e = p.order[w / p.pairs], pr = w % p.pairs;
+    const int b = e / (p.Hm * p.nqt), hm = (e / p.nqt) % p.Hm, qt = e % p.nqt;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      t[s].valid = true;
+      t[s].n = p.count[e];
+      t[s].h0 = (2 * pr + s) * GP;
+      t[s].q0 = qt * BQ;
+      t[s].b = b;
+      t[s].bh_mask = static_cast<size_t>(b) * p.Hm + hm;
+      t[s].lst = p.list + static_cast<size_t>(e) * p.nkt;
+      t[s].cls = p.cls + static_cast<size_t>(e) * p.nkt;
+    }
+  } else {
+    const int qp = w % p.nqp, ht = (w / p.nqp) % p.n_ht, b = w / (p.nqp * p.n_ht);
+    const int hm = p.Hm == 1 ? 0 : ht;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int qt = 2 * qp + s;
+      const size_t e = (static_cast<size_t>(b) * p.Hm + hm) * p.nqt + qt;
+      t[s].valid = qt < p.nqt;
+      t[s].n = t[s].valid ? p.count[e] : 0;
+      t[s].h0 = ht * GP;
+      t[s].q0 = qt * BQ;
+      t[s].b = b;
+      t[s].bh_mask = static_cast<size_t>(b) * p.Hm + hm;
+      t[s].lst = p.list + e * p.nkt;
+      t[s].cls = p.cls + e * p.nkt;
+    }
+  }
+  hkv = t[0].h0 / p.G;
+}
+
+// Walks the union of the two tiles' ascending k-tile lists.
+struct Merge {
+  const int32_t* l0;
+  const int32_t* l1;
+  int n0, n1, i0, i1;
+  bool shared;
+  __device__ __forceinline__ bool next(int& kt, bool& in0, bool& in1) {
+    if (shared) {
+      if (i0 >= n0) return false;
+      kt = l0[i0++];
+      in0 = in1 = true;
+      return true;
+    }
+    const int a = i0 < n0 ? l0[i0] : INT_MAX;
+    const int c = i1 < n1 ? l1[i1] : INT_MAX;
+    if (a == INT_MAX && c == INT_MAX) return false;
+    kt = min(a, c);
+    in0 = a == kt;
+    in1 = c == kt;
+    i0 += in0;
+    i1 += in1;
+    return true;
+  }
+};
+
+__device__ __forceinline__ Merge make_merge(const FwdParams& p, const Tile (&t)[2]) {
+  Merge m;
+  m.l0 = t[0].lst; m.l1 = t[1].lst;
+  m.n0 = t[0].n; m.n1 = t[1].n;
+  m.i0 = m.i1 = 0;
+  m.shared = p.item_kind == 0;
+  return m;
+}
+
+// Snake order over rounds of gridDim.x items: CTA c takes item c in even rounds
+// and item gridDim.x - 1 - c in odd rounds, which evens out LPT-sorted costs.
+__device__ __forceinline__ int item_of_round(int r) {
+  return r * gridDim.x + ((r & 1) ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x);
+}
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
@@ -79,55 +186,52 @@ template <int D, int BK, int GP>
 __global__ void __launch_bounds__(kThreads, 1)
     mfa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = Smem<D, BK>;
+  using C = Cfg<D, BK>;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-  uint8_t* sQ = smem + L::kQ;
-  uint8_t* sK = smem + L::kK;
-  uint8_t* sV = smem + L::kV;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint8_t* sQ = smem + C::kQ;
+  uint8_t* sK = smem + C::kK;
+  uint8_t* sV = smem + C::kV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBar);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + kStagesK;
-  uint64_t* v_full = k_empty + kStagesK;
-  uint64_t* v_empty = v_full + kStagesV;
-  uint64_t* s_full = v_empty + kStagesV;
+  uint64_t* q_empty = q_full + 2;
+  uint64_t* k_full = q_empty + 2;
+  uint64_t* k_empty = k_full + S;
+  uint64_t* v_full = k_empty + S;
+  uint64_t* v_empty = v_full + S;
+  uint64_t* s_full = v_empty + S;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
-  uint64_t* drain = o_done + 1;
-  uint64_t* bnd_full = drain + 1;
-  int4* s_bounds = reinterpret_cast<int4*>(smem + L::kBounds);
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kMisc);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  uint64_t* bnd_full = o_done + 2;  // [2 tiles][2 slots]
+  uint64_t* drain = bnd_full + 4;
+  int4* s_bounds = reinterpret_cast<int4*>(smem + C::kBounds);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // ---- work item -------------------------------------------------------
-  const int w = blockIdx.x;
-  const int ent = p.order[w / p.hpe];
-  const int ht = w % p.hpe;
-  const int b = ent / (p.Hm * p.nqt);
-  const int hm = (ent / p.nqt) % p.Hm;
-  const int qt = ent % p.nqt;
-  const int h0 = (p.Hm == 1) ? ht * GP : hm;
-  const int hkv = h0 / p.G;
-  const int BQ = kRows / GP;
-  const int q0 = qt * BQ;
-  const int n = p.count[ent];
-  const int32_t* lst = p.list + static_cast<size_t>(ent) * p.nkt;
-  const uint8_t* ccls = p.cls + static_cast<size_t>(ent) * p.nkt;
+  const int wg = warp >> 2;
+  const int n_rounds = (p.n_items + gridDim.x - 1) / gridDim.x;
 
   // ---- set-up ----------------------------------------------------------
   if (warp == 0 && lane == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < kStagesK; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
-    for (int s = 0; s < kStagesV; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&p_full[s], kRows); }
-    mbar_init(o_done, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&q_full[t], 1);
+      mbar_init(&q_empty[t], 1);
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], kRows);
+      mbar_init(&o_done[t], 1);
+      mbar_init(&bnd_full[2 * t], kRows);
+      mbar_init(&bnd_full[2 * t + 1], kRows);
+    }
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 2);  // one arrival per tile slot for every k-tile
+    }
     mbar_init(drain, 1);
-    mbar_init(&bnd_full[0], kRows);
-    mbar_init(&bnd_full[1], kRows);
     *s_abort = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_q);
@@ -135,265 +239,372 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_v);
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, L::kTmemCols);
+    tmem_alloc(s_tmem, C::kTmemCols);
     tmem_relinquish();
     tc_fence_before();
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const uint32_t tmem_o = tmem + 2 * BK;
 
-  if (warp == 0) {
+  if (wg == 0) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(kRegsLow));
+   if (warp == 0) {
     // =================== TMA producer ===================
-    if (lane == 0 && n > 0) {
-      mbar_arrive_expect_tx(q_full, L::kQBytes);
+    if (lane == 0) {
+      uint32_t kv_it = 0;
+      int quse[2] = {0, 0};
+      uint32_t k_inflight = 0, v_inflight = 0;  // loads issued (for the abort drain)
+      bool stop = false;
+      for (int r = 0; r < n_rounds && !stop; ++r) {
+        const int w = item_of_round(r);
+        if (w >= p.n_items) continue;
+        Tile t[2];
+        int hkv;
+        decode_item<GP>(p, w, t, hkv);
+        for (int s = 0; s < 2 && !stop; ++s) {
+          if (t[s].n == 0) continue;
+          if (quse[s] > 0 && !mbar_wait(&q_empty[s], (quse[s] - 1) & 1, s_abort)) { stop = true; break; }
+          mbar_arrive_expect_tx(&q_full[s], C::kQBytes);
+          uint8_t* dst = sQ + s * C::kQBytes;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int head = (GP == 2) ? h0 + hh : h0;
-        const int row = (GP == 2) ? q0 : q0 + 64 * hh;
+          for (int hh = 0; hh < 2; ++hh) {
+            const int head = (GP == 2) ? t[s].h0 + hh : t[s].h0;
+            const int row = (GP == 2) ? t[s].q0 : t[s].q0 + 64 * hh;
 #pragma unroll
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(sQ + c * (kRows * 128) + hh * (64 * 128), &tm_q, q_full, c * 64, row, head, b);
-      }
-      int k_issued = 0, v_issued = 0;
-      for (int i = 0; i < n; ++i) {
-        const int kt = lst[i];
-        if (kt < 0 || kt >= p.nkt) {
-          atomicOr(p.err, MFA_DEVERR_MAP);
-          *s_abort = 1;
-          break;
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_4d(dst + c * (kRows * 128) + hh * (64 * 128), &tm_q, &q_full[s], c * 64, row, head, t[s].b);
+          }
+          ++quse[s];
         }
-        const int ks = i % kStagesK;
-        if (i >= kStagesK && !mbar_wait(&k_empty[ks], ((i / kStagesK) - 1) & 1, s_abort)) break;
-        mbar_arrive_expect_tx(&k_full[ks], L::kKVBytes);
+        Merge m = make_merge(p, t);
+        int kt;
+        bool in0, in1;
+        while (!stop && m.next(kt, in0, in1)) {
+          if (kt < 0 || kt >= p.nkt) {
+            atomicOr(p.err, MFA_DEVERR_MAP);
+            *s_abort = 1;
+            stop = true;
+            break;
+          }
+          const int st = kv_it % S;
+          const uint32_t ph = (kv_it / S) & 1;
+          if (kv_it >= S && !mbar_wait(&k_empty[st], ph ^ 1, s_abort)) { stop = true; break; }
+          mbar_arrive_expect_tx(&k_full[st], C::kKVBytes);
 #pragma unroll
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(sK + ks * L::kKVBytes + c * (BK * 128), &tm_k, &k_full[ks], c * 64, kt * BK, hkv, b);
-        k_issued = i + 1;
-        const int vs = i % kStagesV;
-        if (i >= kStagesV && !mbar_wait(&v_empty[vs], ((i / kStagesV) - 1) & 1, s_abort)) break;
-        mbar_arrive_expect_tx(&v_full[vs], L::kKVBytes);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(sK + st * C::kKVBytes + c * (BK * 128), &tm_k, &k_full[st], c * 64, kt * BK, hkv, t[0].b);
+          k_inflight = kv_it + 1;
+          if (kv_it >= S && !mbar_wait(&v_empty[st], ph ^ 1, s_abort)) { stop = true; break; }
+          mbar_arrive_expect_tx(&v_full[st], C::kKVBytes);
 #pragma unroll
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(sV + vs * L::kKVBytes + c * (BK * 128), &tm_v, &v_full[vs], c * 64, kt * BK, hkv, b);
-        v_issued = i + 1;
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(sV + st * C::kKVBytes + c * (BK * 128), &tm_v, &v_full[st], c * 64, kt * BK, hkv, t[0].b);
+          v_inflight = kv_it + 1;
+          ++kv_it;
+        }
       }
       if (*s_abort) {
-        // Let the copies already issued land before the CTA's shared memory goes away.
+        // Let the copies already issued land before shared memory is released.
         volatile int no_abort = 0;
-        mbar_wait(q_full, 0, &no_abort);
-        for (int j = (k_issued > kStagesK ? k_issued - kStagesK : 0); j < k_issued; ++j)
-          mbar_wait(&k_full[j % kStagesK], (j / kStagesK) & 1, &no_abort);
-        for (int j = (v_issued > kStagesV ? v_issued - kStagesV : 0); j < v_issued; ++j)
-          mbar_wait(&v_full[j % kStagesV], (j / kStagesV) & 1, &no_abort);
+        for (int s = 0; s < 2; ++s)
+          if (quse[s] > 0) mbar_wait(&q_full[s], (quse[s] - 1) & 1, &no_abort);
+        for (uint32_t j = (k_inflight > S ? k_inflight - S : 0); j < k_inflight; ++j)
+          mbar_wait(&k_full[j % S], (j / S) & 1, &no_abort);
+        for (uint32_t j = (v_inflight > S ? v_inflight - S : 0); j < v_inflight; ++j)
+          mbar_wait(&v_full[j % S], (j / S) & 1, &no_abort);
       }
     }
   } else if (warp == 1) {
     // =================== MMA issuer ===================
-    if (lane == 0 && n > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kRows, BK, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kRows, D, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      bool ok = mbar_wait(q_full, 0, s_abort);
-      tc_fence_after();
-      for (int i = 0; ok && i <= n; ++i) {
-        if (i < n) {
-          const int ks = i % kStagesK;
-          if (!(ok = mbar_wait(&k_full[ks], (i / kStagesK) & 1, s_abort))) break;
+      uint32_t kv_it = 0;
+      uint32_t pcount[2] = {0, 0};
+      int quse[2] = {0, 0};
+      bool ok = true;
+      for (int r = 0; r < n_rounds && ok; ++r) {
+        const int w = item_of_round(r);
+        if (w >= p.n_items) continue;
+        Tile t[2];
+        int hkv;
+        decode_item<GP>(p, w, t, hkv);
+        bool pending[2] = {false, false}, first_pv[2] = {true, true}, qready[2] = {false, false};
+        int pstage[2] = {0, 0}, nS[2] = {0, 0}, nPV[2] = {0, 0};
+        uint32_t pphase[2] = {0, 0};
+
+        // O_t += P_t V for the tile's pending k-tile.
+        auto issue_pv = [&](int s) -> bool {
+          if (!mbar_wait(&p_full[s], pcount[s] & 1, s_abort)) return false;
+          ++pcount[s];
+          if (!mbar_wait(&v_full[pstage[s]], pphase[s], s_abort)) return false;
           tc_fence_after();
-          const uint32_t d_s = tmem + (i & 1) * BK;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;  // 16 bf16 along K inside the 128-byte row
-            const uint64_t a = sdesc_sw128(q_addr + (kk >> 2) * (kRows * 128) + off, 16, 1024);
-            const uint64_t bd = sdesc_sw128(k_addr + ks * L::kKVBytes + (kk >> 2) * (BK * 128) + off, 16, 1024);
-            umma_ss(d_s, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[i & 1]);
-          umma_commit(&k_empty[ks]);
-        }
-        if (i >= 1) {
-          const int j = i - 1;
-          if (!(ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, s_abort))) break;
-          const int vs = j % kStagesV;
-          if (!(ok = mbar_wait(&v_full[vs], (j / kStagesV) & 1, s_abort))) break;
+          const uint32_t a_p = tmem + s * BK;
+          const uint32_t d_o = tmem + 2 * BK + s * D;
+          // Descriptor start addresses are in 16-byte units in the low bits, so
+          // advancing by a byte offset adds offset >> 4 to the descriptor.
+          const uint64_t vd = sdesc_sw128(v_addr + pstage[s] * C::kKVBytes, BK * 128, 1024);
+#pragma unroll 1
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * (16 * 128 / 16)), idesc_pv,
+                    (first_pv[s] && kk == 0) ? 0u : 1u);
+          // S_t of the next k-tile is issued after this P.V, so its s_full commit
+          // also covers this MMA; o_done is needed only after the tile's last P.V.
+          if (++nPV[s] == t[s].n) umma_commit(&o_done[s]);
+          umma_commit(&v_empty[pstage[s]]);
+          first_pv[s] = false;
+          pending[s] = false;
+          return true;
+        };
+
+        Merge m = make_merge(p, t);
+        int kt;
+        bool in[2];
+        while (ok && m.next(kt, in[0], in[1])) {
+          const int st = kv_it % S;
+          const uint32_t ph = (kv_it / S) & 1;
+          if (!(ok = mbar_wait(&k_full[st], ph, s_abort))) break;
           tc_fence_after();
-          const uint32_t a_p = tmem + (j & 1) * BK;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t bd = sdesc_sw128(v_addr + vs * L::kKVBytes + kk * (16 * 128), BK * 128, 1024);
-            umma_ts(tmem_o, a_p + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int s = 0; s < 2; ++s) {
+            if (pending[s] && !(ok = issue_pv(s))) break;
+            if (in[s]) {
+              if (!qready[s]) {
+                if (!(ok = mbar_wait(&q_full[s], quse[s] & 1, s_abort))) break;
+                tc_fence_after();
+                qready[s] = true;
+              }
+              const uint64_t qd = sdesc_sw128(q_addr + s * C::kQBytes, 16, 1024);
+              const uint64_t kd = sdesc_sw128(k_addr + st * C::kKVBytes, 16, 1024);
+#pragma unroll 1
+              for (int kk = 0; kk < D / 16; ++kk) {
+                // K step of 16 bf16 = 32 bytes inside the 128-byte row; every 4
+                // steps move to the next 64-column chunk of the tile.
+                const uint32_t off = (kk & 3) * 32;
+                const uint64_t a = qd + static_cast<uint64_t>(((kk >> 2) * (kRows * 128) + off) >> 4);
+                const uint64_t bd = kd + static_cast<uint64_t>(((kk >> 2) * (BK * 128) + off) >> 4);
+                umma_ss(tmem + s * BK, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+              }
+              umma_commit(&s_full[s]);
+              pending[s] = true;
+              pstage[s] = st;
+              pphase[s] = ph;
+              if (++nS[s] == t[s].n) umma_commit(&q_empty[s]);  // last read of Q_s in this item
+            } else {
+              mbar_arrive(&v_empty[st]);  // this tile does not read V at this k-tile
+            }
           }
-          umma_commit(o_done);
-          umma_commit(&v_empty[vs]);
+          if (!ok) break;
+          umma_commit(&k_empty[st]);
+          ++kv_it;
         }
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+          if (ok && pending[s]) ok = issue_pv(s);
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+          if (t[s].n > 0) ++quse[s];
       }
+      if (!ok) *s_abort = 1;
       // Wait for every MMA issued here before TMEM can be released.
       umma_commit(drain);
       volatile int no_abort = 0;
       mbar_wait(drain, 0, &no_abort);
     }
-  } else if (warp >= 4) {
+   }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(kRegsHigh));
     // =================== softmax / correction / epilogue ===================
-    const int sw = warp - 4;
+    const int slot = wg - 1;
+    const int sw = warp & 3;
     const int r = sw * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(sw * 32) << 16;
-    const int qi = (GP == 2) ? q0 + (r & 63) : q0 + r;
-    const int head = (GP == 2) ? h0 + (r >> 6) : h0;
+    const uint32_t tmem_s = tmem + slot * BK;
+    const uint32_t tmem_o = tmem + 2 * BK + slot * D;
     const MaskArgs& mk = p.mask;
-    const size_t bh_mask = static_cast<size_t>(b) * p.Hm + hm;
     const bool k_ragged = (p.Nk % BK) != 0;
-
-    float m_run = -INFINITY, l_run = 0.f;
+    int4* my_bounds = s_bounds + slot * 2 * BK;
+    uint64_t* my_bnd = bnd_full + 2 * slot;
+    uint32_t s_cnt = 0, o_cnt = 0, n_bnd = 0;
     bool ok = true;
-    int n_bnd = 0;  // colwise partial tiles staged so far
-    for (int i = 0; i < n; ++i) {
-      const int kt = lst[i];
-      if (kt < 0 || kt >= p.nkt) {
-        if (lane == 0) atomicOr(p.err, MFA_DEVERR_MAP);
-        *s_abort = 1;
-        ok = false;
-        break;
-      }
-      const uint32_t cb = ccls[kt];
-      const bool partial = ((cb & 3u) == 2u) || (k_ragged && kt == p.nkt - 1);
-      const int4* bnd = nullptr;
-      if (partial && mk.kind == MFA_MASK_COLWISE) {
-        // Stage the tile's column bounds in shared memory (double-buffered; a
-        // thread reaching partial tile t+2 has passed tile t+1's barrier, so
-        // every reader of tile t is done with the slot it overwrites).
-        const int slot = n_bnd & 1;
-        int4* dst = s_bounds + slot * BK;
-        if (r < BK) {
-          const int j = kt * BK + r;
-          int4 v = make_int4(0, 0x7fffffff, 0, 0);  // columns past Nk: masked for every row
-          if (j < p.Nk) {
-            const size_t idx = bh_mask * p.Nk + j;
-            v.x = mk.lts ? mk.lts[idx] : 0;
-            v.y = mk.lte ? mk.lte[idx] : 0;
-            v.z = mk.uts ? mk.uts[idx] : 0;
-            v.w = mk.ute ? mk.ute[idx] : 0;
-          }
-          dst[r] = v;
-        }
-        mbar_arrive(&bnd_full[slot]);
-        if (!(ok = warp_all(mbar_wait(&bnd_full[slot], (n_bnd >> 1) & 1, s_abort)))) break;
-        bnd = dst;
-        ++n_bnd;
-      }
-      if (!(ok = warp_all(mbar_wait(&s_full[i & 1], (i >> 1) & 1, s_abort)))) break;
-      tc_fence_after();
 
-      float s[BK];
-      {
-        uint32_t* su = reinterpret_cast<uint32_t*>(s);
-#pragma unroll
-        for (int c = 0; c < BK / 32; ++c)
-          tmem_ld_32x32b_x32(tmem + lane_off + (i & 1) * BK + c * 32,
-                             *reinterpret_cast<uint32_t(*)[32]>(su + c * 32));
-        tmem_ld_wait();
-      }
-      if (partial) {
-        const int jb = kt * BK;
-        if (mk.kind == MFA_MASK_COLWISE) {
-#pragma unroll
-          for (int jj = 0; jj < BK; ++jj) {
-            const int4 v = bnd[jj];
-            const bool masked = (v.x <= qi && qi < v.y) || (v.z <= qi && qi < v.w);
-            if (masked) s[jj] = -INFINITY;
-          }
-        } else if (mk.kind == MFA_MASK_BAND) {
-#pragma unroll
-          for (int jj = 0; jj < BK; ++jj) {
-            const int dj = jb + jj - qi;
-            const bool vis = (jb + jj < p.Nk) && dj >= -mk.pre && dj <= mk.nxt;
-            if (!vis) s[jj] = -INFINITY;
-          }
-        } else {
-          const int qsl = (GP == 2) ? 0 : (r >> 6);
-#pragma unroll
-          for (int jj = 0; jj < BK; ++jj) {
-            const int ksl = jj >> 6;
-            const bool vis = (jb + jj < p.Nk) && (jb + jj <= qi) && ((cb >> (4 + 2 * qsl + ksl)) & 1u);
-            if (!vis) s[jj] = -INFINITY;
-          }
+    for (int rr = 0; rr < n_rounds && ok; ++rr) {
+      const int w = item_of_round(rr);
+      if (w >= p.n_items) continue;
+      Tile tt[2];
+      int hkv;
+      decode_item<GP>(p, w, tt, hkv);
+      const Tile T = slot == 0 ? tt[0] : tt[1];
+      if (!T.valid) continue;
+      const int qi = (GP == 2) ? T.q0 + (r & 63) : T.q0 + r;
+      const int head = (GP == 2) ? T.h0 + (r >> 6) : T.h0;
+      const int n = T.n;
+      float m_run = -INFINITY, l_run = 0.f;
+
+      for (int i = 0; i < n; ++i) {
+        const int kt = T.lst[i];
+        if (kt < 0 || kt >= p.nkt) {
+          if (lane == 0) atomicOr(p.err, MFA_DEVERR_MAP);
+          *s_abort = 1;
+          ok = false;
+          break;
         }
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int jj = 0; jj < BK; ++jj) mx = fmaxf(mx, s[jj]);
-      const float mx_s = mx * p.scale_log2;
-      const bool need = mx_s > m_run + kRescaleThreshold;
-      const float m_new = need ? mx_s : m_run;
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      float sum = 0.f;
-#pragma unroll
-      for (int jj = 0; jj < BK; ++jj) {
-        const float e = ex2_approx(fmaf(s[jj], p.scale_log2, -m_use));
-        s[jj] = e;
-        sum += e;
-      }
-      if (i > 0) {
-        if (!(ok = warp_all(mbar_wait(o_done, (i - 1) & 1, s_abort)))) break;
+        const uint32_t cb = T.cls[kt];
+        const bool partial = ((cb & 3u) == 2u) || (k_ragged && kt == p.nkt - 1);
+        const int4* bnd = nullptr;
+        if (partial && mk.kind == MFA_MASK_COLWISE) {
+          // Stage the tile's column bounds (double-buffered: a thread at partial
+          // tile k+2 has passed tile k+1's barrier, so tile k's readers are done).
+          const int bs = n_bnd & 1;
+          int4* dst = my_bounds + bs * BK;
+          if (r < BK) {
+            const int j = kt * BK + r;
+            int4 v = make_int4(0, 0x7fffffff, 0, 0);  // columns past Nk: masked for every row
+            if (j < p.Nk) {
+              const size_t idx = T.bh_mask * p.Nk + j;
+              v.x = mk.lts ? mk.lts[idx] : 0;
+              v.y = mk.lte ? mk.lte[idx] : 0;
+              v.z = mk.uts ? mk.uts[idx] : 0;
+              v.w = mk.ute ? mk.ute[idx] : 0;
+            }
+            dst[r] = v;
+          }
+          mbar_arrive(&my_bnd[bs]);
+          if (!(ok = warp_all(mbar_wait(&my_bnd[bs], (n_bnd >> 1) & 1, s_abort)))) break;
+          bnd = dst;
+          ++n_bnd;
+        }
+        if (!(ok = warp_all(mbar_wait(&s_full[slot], s_cnt & 1, s_abort)))) break;
+        ++s_cnt;
         tc_fence_after();
-      }
-      const float alpha = need ? ex2_approx(m_run - m_use) : 1.f;
-      l_run = l_run * alpha + sum;
-      m_run = m_new;
-      if (i > 0 && __any_sync(0xffffffffu, need)) {
+
+        float s[BK];
+        {
+          uint32_t sv[BK / 32][32];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(tmem_o + lane_off + c * 32, o);
+          for (int c = 0; c < BK / 32; ++c) tmem_ld_32x32b_x32(tmem_s + lane_off + c * 32, sv[c]);
           tmem_ld_wait();
 #pragma unroll
-          for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
-          tmem_st_32x32b_x32(tmem_o + lane_off + c * 32, o);
+          for (int jj = 0; jj < BK; ++jj) s[jj] = __uint_as_float(sv[jj >> 5][jj & 31]);
+        }
+        if (partial) {
+          const int jb = kt * BK;
+          if (mk.kind == MFA_MASK_COLWISE) {
+            // Visibility bits first (a rolled loop keeps the bound loads from
+            // being hoisted all at once), then one select per column.
+            uint32_t vis[BK / 32];
+#pragma unroll
+            for (int wd = 0; wd < BK / 32; ++wd) {
+              uint32_t bits = 0;
+#pragma unroll 4
+              for (int bb = 0; bb < 32; ++bb) {
+                const int4 v = bnd[wd * 32 + bb];
+                const bool masked = (v.x <= qi && qi < v.y) || (v.z <= qi && qi < v.w);
+                bits |= (masked ? 0u : 1u) << bb;
+              }
+              vis[wd] = bits;
+            }
+#pragma unroll
+            for (int jj = 0; jj < BK; ++jj)
+              if (!((vis[jj >> 5] >> (jj & 31)) & 1u)) s[jj] = -INFINITY;
+          } else if (mk.kind == MFA_MASK_BAND) {
+#pragma unroll
+            for (int jj = 0; jj < BK; ++jj) {
+              const int dj = jb + jj - qi;
+              const bool vis = (jb + jj < p.Nk) && dj >= -mk.pre && dj <= mk.nxt;
+              if (!vis) s[jj] = -INFINITY;
+            }
+          } else {
+            const int qsl = (GP == 2) ? 0 : (r >> 6);
+#pragma unroll
+            for (int jj = 0; jj < BK; ++jj) {
+              const int ksl = jj >> 6;
+              const bool vis = (jb + jj < p.Nk) && (jb + jj <= qi) && ((cb >> (4 + 2 * qsl + ksl)) & 1u);
+              if (!vis) s[jj] = -INFINITY;
+            }
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int jj = 0; jj < BK; ++jj) mx = fmaxf(mx, s[jj]);
+        const float mx_s = mx * p.scale_log2;
+        const bool need = mx_s > m_run + kRescaleThreshold;
+        const float m_new = need ? mx_s : m_run;
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        float sum = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < BK; ++jj) {
+          const float e = ex2_approx(fmaf(s[jj], p.scale_log2, -m_use));
+          s[jj] = e;
+          sum += e;
+        }
+        const float alpha = need ? ex2_approx(m_run - m_use) : 1.f;
+        l_run = l_run * alpha + sum;
+        m_run = m_new;
+        // P (bf16) over S. S_t(i) being complete implies P_t(i-1).V is complete
+        // (MMAs finish in issue order), so S and O of this slot are free here.
+#pragma unroll
+        for (int c = 0; c < BK / 64; ++c) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) pk[u] = pack_bf16x2(s[c * 64 + 2 * u], s[c * 64 + 2 * u + 1]);
+          tmem_st_32x32b_x32(tmem_s + lane_off + c * 32, pk);
+        }
+        if (i > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(tmem_o + lane_off + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+            tmem_st_32x32b_x32(tmem_o + lane_off + c * 32, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[slot]);
+      }
+      if (!ok) break;
+
+      // ---- epilogue of this tile ----
+      // The next item's first P.V into this slot's O waits for this warpgroup's
+      // next P, which is written after these reads, so O needs no other guard.
+      if (n > 0) {
+        if (!(ok = warp_all(mbar_wait(&o_done[slot], o_cnt & 1, s_abort)))) break;
+        ++o_cnt;
+        tc_fence_after();
+      }
+      const bool has = l_run > 0.f;
+      const float inv = has ? 1.f / l_run : 0.f;
+      const bool store = qi < p.Nq;
+      __nv_bfloat16* orow = p.out + static_cast<int64_t>(T.b) * p.os0 + static_cast<int64_t>(head) * p.os1 +
+                            static_cast<int64_t>(qi) * p.os2;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (n > 0) {
+          tmem_ld_32x32b_x32(tmem_o + lane_off + c * 32, o);
+          tmem_ld_wait();
+        }
+        if (store) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            uint4 v;
+            v.x = has ? pack_bf16x2(__uint_as_float(o[8 * g + 0]) * inv, __uint_as_float(o[8 * g + 1]) * inv) : 0u;
+            v.y = has ? pack_bf16x2(__uint_as_float(o[8 * g + 2]) * inv, __uint_as_float(o[8 * g + 3]) * inv) : 0u;
+            v.z = has ? pack_bf16x2(__uint_as_float(o[8 * g + 4]) * inv, __uint_as_float(o[8 * g + 5]) * inv) : 0u;
+            v.w = has ? pack_bf16x2(__uint_as_float(o[8 * g + 6]) * inv, __uint_as_float(o[8 * g + 7]) * inv) : 0u;
+            reinterpret_cast<uint4*>(orow)[c * 4 + g] = v;
+          }
         }
       }
-#pragma unroll
-      for (int c = 0; c < BK / 64; ++c) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) pk[t] = pack_bf16x2(s[c * 64 + 2 * t], s[c * 64 + 2 * t + 1]);
-        tmem_st_32x32b_x32(tmem + lane_off + (i & 1) * BK + c * 32, pk);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[i & 1]);
-    }
-
-    // ---- epilogue ----
-    if (ok && n > 0) {
-      ok = warp_all(mbar_wait(o_done, (n - 1) & 1, s_abort));
-      tc_fence_after();
-    }
-    const bool has = ok && l_run > 0.f;
-    const float inv = has ? 1.f / l_run : 0.f;
-    const bool store = qi < p.Nq;
-    __nv_bfloat16* orow = p.out + static_cast<int64_t>(b) * p.os0 + static_cast<int64_t>(head) * p.os1 +
-                          static_cast<int64_t>(qi) * p.os2;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t o[32] = {};
-      if (ok && n > 0) {
-        tmem_ld_32x32b_x32(tmem_o + lane_off + c * 32, o);
-        tmem_ld_wait();
-      }
-      uint32_t pk[16];
-#pragma unroll
-      for (int t = 0; t < 16; ++t)
-        pk[t] = has ? pack_bf16x2(__uint_as_float(o[2 * t]) * inv, __uint_as_float(o[2 * t + 1]) * inv) : 0u;
       if (store) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        const float lse = has ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+        p.lse[(static_cast<size_t>(T.b) * p.Hq + head) * p.Nq + qi] = lse;
       }
-    }
-    if (store) {
-      const float lse = has ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
-      p.lse[(static_cast<size_t>(b) * p.Hq + head) * p.Nq + qi] = lse;
     }
     if (!ok && lane == 0) atomicOr(p.err, MFA_DEVERR_TIMEOUT);
   }
@@ -401,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, L::kTmemCols);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -448,18 +659,28 @@ mfa_status check_tensor(const mfa_tensor* t) {
   return MFA_OK;
 }
 
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
 template <int D, int BK, int GP>
 mfa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
-                  int n_items, cudaStream_t s) {
-  using L = Smem<D, BK>;
+                  cudaStream_t s) {
+  using C = Cfg<D, BK>;
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(mfa_fwd_kernel<D, BK, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) !=
+    if (cudaFuncSetAttribute(mfa_fwd_kernel<D, BK, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) !=
         cudaSuccess)
       return MFA_ERR_CUDA;
     attr_set = true;
   }
-  mfa_fwd_kernel<D, BK, GP><<<n_items, kThreads, L::kAlloc, s>>>(mq, mk, mv, p);
+  const int sms = sm_count();
+  if (sms <= 0) return MFA_ERR_CUDA;
+  const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: at most one CTA per SM
+  mfa_fwd_kernel<D, BK, GP><<<grid, kThreads, C::kAlloc, s>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
 }
 
@@ -498,7 +719,24 @@ extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   p.B = static_cast<int32_t>(q->B); p.Hq = static_cast<int32_t>(q->H); p.Hkv = static_cast<int32_t>(k->H);
   p.G = G; p.Hm = mask->Hm; p.Nq = static_cast<int32_t>(q->N); p.Nk = static_cast<int32_t>(k->N);
   p.nqt = map->nqt; p.nkt = map->nkt;
-  p.hpe = mask->Hm == 1 ? p.Hq / GP : 1;
+  // Work items pair two query tiles that read the same key/value head: two head
+  // tiles of one group when the mask is shared and the group holds an even
+  // number of head tiles (kind 0, same list), else two consecutive query tiles
+  // of one head tile (kind 1, union of the two lists).
+  const int tiles_per_group = G / GP;
+  int64_t n_items64;
+  if (mask->Hm == 1 && tiles_per_group % 2 == 0) {
+    p.item_kind = 0;
+    p.pairs = p.Hq / GP / 2;
+    p.n_ht = 0; p.nqp = 0;
+    n_items64 = static_cast<int64_t>(p.B) * p.nqt * p.pairs;
+  } else {
+    p.item_kind = 1;
+    p.pairs = 0;
+    p.n_ht = p.Hq / GP;
+    p.nqp = (p.nqt + 1) / 2;
+    n_items64 = static_cast<int64_t>(p.B) * p.n_ht * p.nqp;
+  }
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(q->D)));
   p.mask = mask_args(mask);
   p.cls = map->tile_class; p.list = map->tile_list; p.count = map->tile_count; p.order = map->order;
@@ -506,10 +744,9 @@ extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   p.os0 = out->stride[0]; p.os1 = out->stride[1]; p.os2 = out->stride[2];
   p.lse = lse;
   p.err = map->err;
-  const int64_t n_items64 = static_cast<int64_t>(p.B) * p.Hm * p.nqt * p.hpe;
   if (n_items64 <= 0) return MFA_OK;
   if (n_items64 > 0x7fffffff) return MFA_ERR_UNSUPPORTED;
-  const int n_items = static_cast<int>(n_items64);
+  p.n_items = static_cast<int32_t>(n_items64);
 
   // With Nk == 0 every list is empty and the K/V maps are never read.
   CUtensorMap mq, mk, mv;
@@ -519,8 +756,8 @@ extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   if (k->N > 0 && (!make_map(&mk, k, map->block_k) || !make_map(&mv, v, map->block_k))) return MFA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int D = static_cast<int>(q->D), BK = map->block_k;
-  if (D == 128 && BK == 128) return GP == 2 ? launch<128, 128, 2>(mq, mk, mv, p, n_items, s) : launch<128, 128, 1>(mq, mk, mv, p, n_items, s);
-  if (D == 128 && BK == 64) return GP == 2 ? launch<128, 64, 2>(mq, mk, mv, p, n_items, s) : launch<128, 64, 1>(mq, mk, mv, p, n_items, s);
-  if (D == 64 && BK == 128) return GP == 2 ? launch<64, 128, 2>(mq, mk, mv, p, n_items, s) : launch<64, 128, 1>(mq, mk, mv, p, n_items, s);
-  return GP == 2 ? launch<64, 64, 2>(mq, mk, mv, p, n_items, s) : launch<64, 64, 1>(mq, mk, mv, p, n_items, s);
+  if (D == 128 && BK == 128) return GP == 2 ? launch<128, 128, 2>(mq, mk, mv, p, s) : launch<128, 128, 1>(mq, mk, mv, p, s);
+  if (D == 128 && BK == 64) return GP == 2 ? launch<128, 64, 2>(mq, mk, mv, p, s) : launch<128, 64, 1>(mq, mk, mv, p, s);
+  if (D == 64 && BK == 128) return GP == 2 ? launch<64, 128, 2>(mq, mk, mv, p, s) : launch<64, 128, 1>(mq, mk, mv, p, s);
+  return GP == 2 ? launch<64, 64, 2>(mq, mk, mv, p, s) : launch<64, 64, 1>(mq, mk, mv, p, s);
 }
