@@ -53,10 +53,10 @@ constexpr int kRows = 128;  // MMA M: query rows per tile
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 =
-// 64512); WG0 drops to 56 and the two softmax warpgroups rise to 224:
-// 128 x 56 + 256 x 224 = 64512.
-constexpr int kRegsLow = 56;
-constexpr int kRegsHigh = 224;
+// 64512); WG0 drops to 104 (the unrolled MMA issue must not spill) and the two
+// softmax warpgroups rise to 200: 128 x 104 + 256 x 200 = 64512.
+constexpr int kRegsLow = 104;
+constexpr int kRegsHigh = 200;
 
 struct FwdParams {
   int32_t B, Hq, Hkv, G, Hm, Nq, Nk, nqt, nkt;
@@ -181,6 +181,31 @@ __device__ __forceinline__ int item_of_round(int r) {
 }
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+// Bits [a, b) of a 32-bit word, with a and b clamped to [0, 32].
+__device__ __forceinline__ uint32_t rows_in_interval(int a, int b) {
+  a = max(a, 0);
+  b = min(b, 32);
+  if (a >= b) return 0u;
+  return static_cast<uint32_t>(((1ull << b) - 1ull) & ~((1ull << a) - 1ull));
+}
+
+// Transpose a 32x32 bit matrix held one row per lane (bit l of lane j's word
+// is entry (j, l)): afterwards bit j of lane l's word is entry (j, l). Five
+// butterfly stages; at distance d each lane keeps the half of its word whose
+// bit index agrees with its own lane bit d and takes the other half from lane
+// l ^ d, shifted by d.
+__device__ __forceinline__ uint32_t transpose32_warp(uint32_t x, int lane) {
+  const uint32_t masks[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+  for (int st = 0; st < 5; ++st) {
+    const int d = 16 >> st;
+    const uint32_t m = masks[st];
+    const uint32_t y = __shfl_xor_sync(0xffffffffu, x, d);
+    x = (lane & d) ? ((x & ~m) | ((y & ~m) >> d)) : ((x & m) | ((y & m) << d));
+  }
+  return x;
+}
 
 template <int D, int BK, int GP>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -345,11 +370,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t d_o = tmem + 2 * BK + s * D;
           // Descriptor start addresses are in 16-byte units in the low bits, so
           // advancing by a byte offset adds offset >> 4 to the descriptor.
+          // The MMAs are issued fully unrolled: a rolled issue loop costs about
+          // twice the MMA's own 64 cycles per instruction.
           const uint64_t vd = sdesc_sw128(v_addr + pstage[s] * C::kKVBytes, BK * 128, 1024);
-#pragma unroll 1
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * (16 * 128 / 16)), idesc_pv,
-                    (first_pv[s] && kk == 0) ? 0u : 1u);
+          umma_ts(d_o, a_p, vd, idesc_pv, first_pv[s] ? 0u : 1u);
+#pragma unroll
+          for (int kk = 1; kk < BK / 16; ++kk)
+            umma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * (16 * 128 / 16)), idesc_pv, 1u);
           // S_t of the next k-tile is issued after this P.V, so its s_full commit
           // also covers this MMA; o_done is needed only after the tile's last P.V.
           if (++nPV[s] == t[s].n) umma_commit(&o_done[s]);
@@ -378,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               const uint64_t qd = sdesc_sw128(q_addr + s * C::kQBytes, 16, 1024);
               const uint64_t kd = sdesc_sw128(k_addr + st * C::kKVBytes, 16, 1024);
-#pragma unroll 1
+#pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
                 // K step of 16 bf16 = 32 bytes inside the 128-byte row; every 4
                 // steps move to the next 64-column chunk of the tile.
@@ -492,23 +519,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (partial) {
           const int jb = kt * BK;
           if (mk.kind == MFA_MASK_COLWISE) {
-            // Visibility bits first (a rolled loop keeps the bound loads from
-            // being hoisted all at once), then one select per column.
-            uint32_t vis[BK / 32];
+            // The warp's 32 lanes hold 32 consecutive queries from qbase. Lane j
+            // turns column (32c + j)'s two intervals into one word of masked
+            // rows (bit l = query qbase + l), then a 32x32 bit transpose across
+            // the warp gives every lane its own row's bits for those columns.
+            const int qbase = qi - lane;
+            uint32_t mrow[BK / 32];
 #pragma unroll
-            for (int wd = 0; wd < BK / 32; ++wd) {
-              uint32_t bits = 0;
-#pragma unroll 4
-              for (int bb = 0; bb < 32; ++bb) {
-                const int4 v = bnd[wd * 32 + bb];
-                const bool masked = (v.x <= qi && qi < v.y) || (v.z <= qi && qi < v.w);
-                bits |= (masked ? 0u : 1u) << bb;
-              }
-              vis[wd] = bits;
+            for (int c = 0; c < BK / 32; ++c) {
+              const int4 v = bnd[c * 32 + lane];
+              uint32_t w = rows_in_interval(v.x - qbase, v.y - qbase) | rows_in_interval(v.z - qbase, v.w - qbase);
+              mrow[c] = transpose32_warp(w, lane);
             }
 #pragma unroll
             for (int jj = 0; jj < BK; ++jj)
-              if (!((vis[jj >> 5] >> (jj & 31)) & 1u)) s[jj] = -INFINITY;
+              if ((mrow[jj >> 5] >> (jj & 31)) & 1u) s[jj] = -INFINITY;
           } else if (mk.kind == MFA_MASK_BAND) {
 #pragma unroll
             for (int jj = 0; jj < BK; ++jj) {

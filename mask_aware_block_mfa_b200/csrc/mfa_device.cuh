@@ -31,6 +31,27 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x on the FMA/ALU pipes instead of the MUFU unit. Cody and Waite's range
+// reduction: x = j + f with j = round(x) (adding 1.5 * 2^23 leaves round(x) in
+// the low mantissa bits) and f in [-1/2, 1/2]; 2^f from the degree-3 polynomial
+// of minimum relative error on [-1/2, 1/2] (Remez exchange, coefficients from
+// csrc/exp2_poly_fit.py, max relative error 7.5e-5 in float32); 2^j is added
+// to the exponent field. Exactly 0 below -125, so masked (-inf) scores give 0.
+constexpr float kExp2C0 = 0x1.fff692p-1f;
+constexpr float kExp2C1 = 0x1.62f31ap-1f;
+constexpr float kExp2C2 = 0x1.f0de1ap-3f;
+constexpr float kExp2C3 = 0x1.c3f76p-5f;
+
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float xc = fmaxf(x, -125.f);
+  const float t = __fadd_rn(xc, 12582912.f);
+  const float j = __fsub_rn(t, 12582912.f);
+  const float f = __fsub_rn(xc, j);
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  const uint32_t bits = __float_as_uint(p) + (__float_as_uint(t) << 23);
+  return x < -125.f ? 0.f : __uint_as_float(bits);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   // cvt.rn.bf16x2.f32 d, a, b puts a in the upper and b in the lower half.
