@@ -159,15 +159,17 @@ mfa_status mfa_tile_map_init(mfa_tile_map* map, void* device_buf, size_t bytes,
 mfa_status mfa_build_tile_map(const mfa_mask_desc* mask, mfa_tile_map* map, void* stream);
 
 /* Attention forward pass on `stream`.
- *   q   [B, Hq, Nq, D], k and v [B, Hkv, Nk, D], out [B, Hq, Nq, D]: dtype
- *       MFA_BF16 (MFA_F32 is rejected as UNSUPPORTED), D in {64, 128},
- *       Hq % Hkv == 0 (query head h reads key/value head h / (Hq/Hkv)),
+ *   q   [B, Hq, Nq, D], k and v [B, Hkv, Nk, D], out [B, Hq, Nq, D], all of one
+ *       dtype, D in {64, 128}: MFA_BF16 runs on the bf16 tensor cores; MFA_F32
+ *       runs in fp32 on the CUDA cores (tf32 tensor-core scores would move lse
+ *       by ~2e-3) and writes fp32 out. Hq % Hkv == 0: query head h reads
+ *       key/value head h / (Hq/Hkv).
  *       stride[3] == 1, other strides and the base address 16-byte aligned.
  *   mask  description with mask->map built from it by mfa_build_tile_map
  *         (same kind and shape); Hm must be 1 or Hq.
  *   lse   float32 [B, Hq, Nq] contiguous, natural-log log-sum-exp per row.
- * Query tiles pack heads: block_q == 128 puts 128 queries of one head in a
- * tile; block_q == 64 puts 64 queries of two heads of one key/value group in
+ * bf16 query tiles pack heads: block_q == 128 puts 128 queries of one head in
+ * a tile; block_q == 64 puts 64 queries of two heads of one key/value group in
  * a tile and needs Hm == 1 and an even Hq/Hkv. block_k is 64 or 128.
  * Rows with no visible key get out = 0 and lse = -inf. */
 mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v,

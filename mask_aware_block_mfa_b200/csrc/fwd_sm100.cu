@@ -726,7 +726,6 @@ extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   if ((st = check_map_matches(mask, map)) != MFA_OK) return st;
   if (map->kind != mask->kind) return MFA_ERR_SHAPE_MISMATCH;
   if (q->dtype != k->dtype || q->dtype != v->dtype || out->dtype != q->dtype) return MFA_ERR_INVALID_ARG;
-  if (q->dtype != MFA_BF16) return MFA_ERR_UNSUPPORTED;
   if (k->B != q->B || v->B != q->B || out->B != q->B) return MFA_ERR_SHAPE_MISMATCH;
   if (k->H != v->H || k->N != v->N || k->D != q->D || v->D != q->D) return MFA_ERR_SHAPE_MISMATCH;
   if (out->H != q->H || out->N != q->N || out->D != q->D) return MFA_ERR_SHAPE_MISMATCH;
@@ -735,6 +734,7 @@ extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   if (mask->Hm != 1 && mask->Hm != q->H) return MFA_ERR_SHAPE_MISMATCH;
   if (q->D != 64 && q->D != 128) return MFA_ERR_UNSUPPORTED;
   if (q->N > (int64_t(1) << 30) || k->N > (int64_t(1) << 30) || q->H > 65535) return MFA_ERR_UNSUPPORTED;
+  if (q->dtype == MFA_F32) return launch_fwd_f32(q, k, v, mask, map, out, lse, static_cast<cudaStream_t>(stream));
   const int G = static_cast<int>(q->H / k->H);
   const int GP = map->block_q == 64 ? 2 : 1;
   if (GP == 2 && (mask->Hm != 1 || G % 2 != 0)) return MFA_ERR_UNSUPPORTED;

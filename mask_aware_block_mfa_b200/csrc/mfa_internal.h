@@ -92,4 +92,9 @@ inline mfa_status check_map_matches(const mfa_mask_desc* d, const mfa_tile_map* 
   return MFA_OK;
 }
 
+// fp32 inputs: the same tile map walked by an fp32 CUDA-core kernel
+// (fwd_f32_simt.cu). Arguments are already validated by mfa_fwd.
+mfa_status launch_fwd_f32(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v, const mfa_mask_desc* mask,
+                          const mfa_tile_map* map, const mfa_tensor* out, float* lse, cudaStream_t s);
+
 }  // namespace mfa

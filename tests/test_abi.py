@@ -136,7 +136,6 @@ def test_fwd_rejects_bad_arguments_on_host(lib):
     q32 = _fake_tensor(1, 8, 512, 128, dtype=B.MFA_F32)
     o32 = _fake_tensor(1, 8, 512, 128, dtype=B.MFA_F32)
     k32, v32 = _fake_tensor(1, 2, 512, 128, dtype=B.MFA_F32), _fake_tensor(1, 2, 512, 128, dtype=B.MFA_F32)
-    assert _fwd(lib, q32, k32, v32, d, o32) == B.MFA_ERR_UNSUPPORTED          # fp32 not implemented
     assert _fwd(lib, q32, k, v, d, o) == B.MFA_ERR_INVALID_ARG                # mixed dtypes
     assert _fwd(lib, _fake_tensor(1, 8, 512, 96), _fake_tensor(1, 2, 512, 96), _fake_tensor(1, 2, 512, 96), d,
                 _fake_tensor(1, 8, 512, 96)) == B.MFA_ERR_UNSUPPORTED         # head dim 96

@@ -20,13 +20,13 @@ from .gpu_util import compare_attention, compare_map, oracle_rows, run_gpu, samp
 pytestmark = pytest.mark.gpu
 
 
-def small_problem(mask, Hq, Hkv, d, seed, Nq=None, Nk=None):
+def small_problem(mask, Hq, Hkv, d, seed, Nq=None, Nk=None, dtype=torch.bfloat16):
     Nq = mask.Nq if Nq is None else Nq
     Nk = mask.Nk if Nk is None else Nk
     g = torch.Generator().manual_seed(seed)
-    q = torch.randn(mask.B, Hq, Nq, d, generator=g).to(torch.bfloat16)
-    k = torch.randn(mask.B, Hkv, Nk, d, generator=g).to(torch.bfloat16)
-    v = torch.randn(mask.B, Hkv, Nk, d, generator=g).to(torch.bfloat16)
+    q = torch.randn(mask.B, Hq, Nq, d, generator=g).to(dtype)
+    k = torch.randn(mask.B, Hkv, Nk, d, generator=g).to(dtype)
+    v = torch.randn(mask.B, Hkv, Nk, d, generator=g).to(dtype)
     return W.Problem("small", q, k, v, mask, seed)
 
 
@@ -60,6 +60,36 @@ def test_fwd_small_all_rows(name, mask, Hq, Hkv, d, blocks):
     prob = small_problem(mask, Hq, Hkv, d, seed=zlib.crc32(name.encode()) % 1000)
     for bq, bk in blocks:
         check_full(prob, bq, bk)
+
+
+FP32_CASES = [
+    # fp32 inputs are computed in fp32 on the CUDA cores; output is fp32
+    ("doc_fp32", W.make_mask("doc8k", N=1024), 4, 2, [(64, 128), (128, 64), (128, 128)]),
+    ("ragged_fp32", W.make_mask("tiny_doc_fp32", N=700), 2, 2, [(128, 64), (128, 128)]),
+    ("band_fp32", W.band(1, 600, 100, -5), 2, 1, [(64, 64), (128, 128)]),
+    ("blocksel_fp32", W.random_blocksel(np.random.default_rng(3), 1, 640, 640, 4), 2, 2, [(128, 64)]),
+]
+
+
+@pytest.mark.parametrize("name,mask,Hq,Hkv,blocks", FP32_CASES, ids=[c[0] for c in FP32_CASES])
+def test_fwd_fp32_all_rows(name, mask, Hq, Hkv, blocks):
+    prob = small_problem(mask, Hq, Hkv, 64, seed=zlib.crc32(name.encode()) % 1000, dtype=torch.float32)
+    for bq, bk in blocks:
+        out, lse, arrays, err = run_gpu(prob, bq, bk)
+        assert err == 0
+        ref_out, ref_lse = oracle_rows(prob, None)
+        compare_attention(out, lse, ref_out, ref_lse)
+
+
+def test_fwd_fp32_d128_and_per_head_masks():
+    rng = np.random.default_rng(12)
+    mask = W.random_colwise(rng, 1, 3, 300, 280)
+    prob = small_problem(mask, 3, 1, 128, seed=1, Nq=300, Nk=280, dtype=torch.float32)
+    for bq, bk in [(64, 128), (128, 64)]:
+        out, lse, _, err = run_gpu(prob, bq, bk)
+        assert err == 0
+        ref_out, ref_lse = oracle_rows(prob, None)
+        compare_attention(out, lse, ref_out, ref_lse)
 
 
 def test_fwd_rectangular_nq_ne_nk():
@@ -104,8 +134,8 @@ def test_fwd_zero_query_closed_form():
 
 
 # Full-size named workloads in the benchmark's launch configuration.
-FULL = [("doc8k", 64, 128), ("shared_question8k", 64, 128), ("band16k", 128, 128), ("band16k_neg", 128, 128),
-        ("doc32k", 64, 128), ("blocksel32k", 64, 64)]
+FULL = [("tiny_doc_fp32", 128, 64), ("doc8k", 64, 128), ("shared_question8k", 64, 128), ("band16k", 128, 128),
+        ("band16k_neg", 128, 128), ("doc32k", 64, 128), ("blocksel32k", 64, 64)]
 
 
 @pytest.mark.parametrize("name,bq,bk", FULL, ids=[f[0] for f in FULL])
