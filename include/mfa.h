@@ -100,8 +100,13 @@ typedef struct {
  *   tile_count int32 [B, Hm, nqt].
  *   order      int32 [B*Hm*nqt] flat (b, hm, qt) sorted by count, largest
  *              first, ties by index (the forward pass's work order).
- *   err        uint32 device error word (MFA_DEVERR_* bits), cleared by
- *              mfa_build_tile_map, set by it and by mfa_fwd.
+ *   err        uint32 [4]: err[0] is the device error word (MFA_DEVERR_*
+ *              bits), set by mfa_build_tile_map and mfa_fwd; err[1] and
+ *              err[2] are mfa_fwd's work counters (the next work item and the
+ *              number of finished CTAs), left at zero after every call. All
+ *              four are cleared by mfa_build_tile_map. Because of the
+ *              counters, mfa_fwd calls that share one map must not overlap on
+ *              the GPU (issue them on one stream, or order the streams).
  * Class rule for COLWISE / BAND with r0 = qt*block_q, r1 = min(r0+block_q, Nq):
  *   SKIP    if (LTSmax <= r0 && LTEmin >= r1) || (UTSmax <= r0 && UTEmin >= r1)
  *   FULL    else if (LTSmin >= r1 || LTEmax <= r0) && (UTSmin >= r1 || UTEmax <= r0)

@@ -71,7 +71,10 @@ struct FwdParams {
   int64_t os0, os1, os2;
   float* lse;
   uint32_t* err;
+  uint32_t* sched;  // [0] next work item, [1] CTAs finished (map scratch words)
 };
+
+constexpr int kRing = 4;  // decoded work items in flight from the producer to the other roles
 
 template <int D, int BK>
 struct Cfg {
@@ -84,10 +87,11 @@ struct Cfg {
   static constexpr int kV = kK + kStages * kKVBytes;
   static constexpr int kBar = kV + kStages * kKVBytes;
   // q_full[2] q_empty[2] k_full[S] k_empty[S] v_full[S] v_empty[S] s_full[2] p_full[2]
-  // o_done[2] bnd[2][2] drain
-  static constexpr int kNumBars = 4 + 4 * kStages + 6 + 4 + 1;
+  // o_done[2] bnd[2][2] drain sched_full[kRing] sched_empty[kRing]
+  static constexpr int kNumBars = 4 + 4 * kStages + 6 + 4 + 1 + 2 * kRing;
   static constexpr int kBounds = kBar + ((kNumBars * 8 + 15) / 16) * 16;  // int4 [2 tiles][2 slots][BK]
-  static constexpr int kMisc = kBounds + 4 * BK * 16;
+  static constexpr int kRingOff = kBounds + 4 * BK * 16;                 // WorkItem [kRing]
+  static constexpr int kMisc = kRingOff + kRing * 128;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
   static constexpr int kTmemCols = (2 * BK + 2 * D) <= 256 ? 256 : 512;
@@ -102,6 +106,14 @@ struct Tile {
   const int32_t* lst;
   const uint8_t* cls;
 };
+
+// One decoded work item as the producer publishes it to the MMA and softmax roles.
+struct WorkItem {
+  int32_t w;    // item index, -1 = no more work
+  int32_t hkv;
+  Tile t[2];
+};
+static_assert(sizeof(WorkItem) <= 128, "ring slot size");
 
 template <int GP>
 __device__ __forceinline__ void decode_item(const FwdParams& p, int w, Tile (&t)[2], int& hkv) {
@@ -174,12 +186,6 @@ __device__ __forceinline__ Merge make_merge(const FwdParams& p, const Tile (&t)[
   return m;
 }
 
-// Snake order over rounds of gridDim.x items: CTA c takes item c in even rounds
-// and item gridDim.x - 1 - c in odd rounds, which evens out LPT-sorted costs.
-__device__ __forceinline__ int item_of_round(int r) {
-  return r * gridDim.x + ((r & 1) ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x);
-}
-
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 // Bits [a, b) of a 32-bit word, with a and b clamped to [0, 32].
@@ -231,13 +237,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_done = p_full + 2;
   uint64_t* bnd_full = o_done + 2;  // [2 tiles][2 slots]
   uint64_t* drain = bnd_full + 4;
+  uint64_t* sched_full = drain + 1;
+  uint64_t* sched_empty = sched_full + kRing;
   int4* s_bounds = reinterpret_cast<int4*>(smem + C::kBounds);
+  WorkItem* ring = reinterpret_cast<WorkItem*>(smem + C::kRingOff);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wg = warp >> 2;
-  const int n_rounds = (p.n_items + gridDim.x - 1) / gridDim.x;
 
   // ---- set-up ----------------------------------------------------------
   if (warp == 0 && lane == 0) {
@@ -257,6 +265,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_empty[s], 2);  // one arrival per tile slot for every k-tile
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&sched_full[i], 1);
+      mbar_init(&sched_empty[i], 1 + 8);  // the MMA thread and one lane of each softmax warp
+    }
     *s_abort = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_q);
@@ -281,12 +293,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       int quse[2] = {0, 0};
       uint32_t k_inflight = 0, v_inflight = 0;  // loads issued (for the abort drain)
       bool stop = false;
-      for (int r = 0; r < n_rounds && !stop; ++r) {
-        const int w = item_of_round(r);
-        if (w >= p.n_items) continue;
-        Tile t[2];
-        int hkv;
-        decode_item<GP>(p, w, t, hkv);
+      // Work items are handed out dynamically in LPT order: an idle CTA takes
+      // the next one. The producer decodes it once and publishes it.
+      for (int it = 0; !stop; ++it) {
+        const int rs = it % kRing;
+        if (it >= kRing && !mbar_wait(&sched_empty[rs], ((it / kRing) - 1) & 1, s_abort)) break;
+        const uint32_t wu = atomicAdd(&p.sched[0], 1u);
+        WorkItem info;
+        info.w = wu < static_cast<uint32_t>(p.n_items) ? static_cast<int>(wu) : -1;
+        info.hkv = 0;
+        if (info.w >= 0) decode_item<GP>(p, info.w, info.t, info.hkv);
+        ring[rs] = info;
+        mbar_arrive(&sched_full[rs]);
+        if (info.w < 0) break;
+        const Tile (&t)[2] = info.t;
+        const int hkv = info.hkv;
         for (int s = 0; s < 2 && !stop; ++s) {
           if (t[s].n == 0) continue;
           if (quse[s] > 0 && !mbar_wait(&q_empty[s], (quse[s] - 1) & 1, s_abort)) { stop = true; break; }
@@ -350,12 +371,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pcount[2] = {0, 0};
       int quse[2] = {0, 0};
       bool ok = true;
-      for (int r = 0; r < n_rounds && ok; ++r) {
-        const int w = item_of_round(r);
-        if (w >= p.n_items) continue;
-        Tile t[2];
-        int hkv;
-        decode_item<GP>(p, w, t, hkv);
+      for (int it = 0; ok; ++it) {
+        const int rs = it % kRing;
+        if (!(ok = mbar_wait(&sched_full[rs], (it / kRing) & 1, s_abort))) break;
+        const WorkItem info = ring[rs];
+        mbar_arrive(&sched_empty[rs]);
+        if (info.w < 0) break;
+        const Tile (&t)[2] = info.t;
         bool pending[2] = {false, false}, first_pv[2] = {true, true}, qready[2] = {false, false};
         int pstage[2] = {0, 0}, nS[2] = {0, 0}, nPV[2] = {0, 0};
         uint32_t pphase[2] = {0, 0};
@@ -457,13 +479,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t s_cnt = 0, o_cnt = 0, n_bnd = 0;
     bool ok = true;
 
-    for (int rr = 0; rr < n_rounds && ok; ++rr) {
-      const int w = item_of_round(rr);
-      if (w >= p.n_items) continue;
-      Tile tt[2];
-      int hkv;
-      decode_item<GP>(p, w, tt, hkv);
-      const Tile T = slot == 0 ? tt[0] : tt[1];
+    for (int it = 0; ok; ++it) {
+      const int rs = it % kRing;
+      if (!(ok = warp_all(mbar_wait(&sched_full[rs], (it / kRing) & 1, s_abort)))) break;
+      const WorkItem info = ring[rs];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sched_empty[rs]);
+      if (info.w < 0) break;
+      const Tile T = slot == 0 ? info.t[0] : info.t[1];
       if (!T.valid) continue;
       const int qi = (GP == 2) ? T.q0 + (r & 63) : T.q0 + r;
       const int head = (GP == 2) ? T.h0 + (r >> 6) : T.h0;
@@ -635,6 +658,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   __syncthreads();
+  if (threadIdx.x == 0) {
+    // The producer (this thread) took its last item before this point; the CTA
+    // that finishes last resets the scheduling words for the next launch.
+    __threadfence();
+    if (atomicAdd(&p.sched[1], 1u) == gridDim.x - 1) {
+      atomicExch(&p.sched[0], 0u);
+      atomicExch(&p.sched[1], 0u);
+      __threadfence();
+    }
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
@@ -769,6 +802,7 @@ extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   p.os0 = out->stride[0]; p.os1 = out->stride[1]; p.os2 = out->stride[2];
   p.lse = lse;
   p.err = map->err;
+  p.sched = map->err + 1;
   if (n_items64 <= 0) return MFA_OK;
   if (n_items64 > 0x7fffffff) return MFA_ERR_UNSUPPORTED;
   p.n_items = static_cast<int32_t>(n_items64);

@@ -33,7 +33,7 @@ inline bool map_layout(int32_t B, int32_t Hm, int32_t Nq, int32_t Nk, int32_t bq
   L->tile_list = off;  off = align256(off + bh * nqt * nkt * sizeof(int32_t));
   L->tile_count = off; off = align256(off + bh * nqt * sizeof(int32_t));
   L->order = off;      off = align256(off + bh * nqt * sizeof(int32_t));
-  L->err = off;        off = align256(off + sizeof(uint32_t));
+  L->err = off;        off = align256(off + 4 * sizeof(uint32_t));  // error word + 2 scheduling words
   L->total = off;
   return true;
 }

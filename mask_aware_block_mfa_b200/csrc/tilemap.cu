@@ -276,7 +276,7 @@ extern "C" mfa_status mfa_build_tile_map(const mfa_mask_desc* mask, mfa_tile_map
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const MaskArgs m = mask_args(mask);
   map->kind = mask->kind;
-  if (cudaMemsetAsync(map->err, 0, sizeof(uint32_t), s) != cudaSuccess) return MFA_ERR_CUDA;
+  if (cudaMemsetAsync(map->err, 0, 4 * sizeof(uint32_t), s) != cudaSuccess) return MFA_ERR_CUDA;
   const int BH = mask->B * mask->Hm;
   if (map->nkt > 0) {
     k_tile_minmax<<<dim3(map->nkt, BH), map->block_k, 0, s>>>(m, map->block_k, map->nkt, map->kminmax,
