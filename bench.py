@@ -220,13 +220,9 @@ def main():
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev_f0=None, ev_f1=None):
-        att.build(stream)
-        if ev_f0 is not None:
-            ev_f0.record(stream)
-        att(q, k, v, out, lse, stream)
-        if ev_f1 is not None:
-            ev_f1.record(stream)
+    def step():
+        att.build()
+        att(q, k, v, out, lse)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -235,24 +231,46 @@ def main():
     if B.device_status(att.tmap, stream) != 0:
         raise RuntimeError("device error word set during warm-up")
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # One step (map build + forward) and the forward alone, captured as CUDA
+    # graphs so the timed region measures device work, not host launch latency.
+    g_step, g_fwd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g_step, stream=cap):
+            step()
+        with torch.cuda.graph(g_fwd, stream=cap):
+            att(q, k, v, out, lse)
+    stream.wait_stream(cap)
+    for _ in range(args.warmup):
+        g_step.replay()
+        g_fwd.replay()
+    torch.cuda.synchronize(dev)
+
+    def timed(graph):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for e0, e1 in evs:
+            flush.fill_(1.0)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+        return evs
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
         time.sleep(0.3)
-        for e0, f0, f1, e1 in ev:
-            flush.fill_(1.0)
-            e0.record(stream)
-            step(f0, f1)
-            e1.record(stream)
+        ev_step = timed(g_step)
+        ev_fwd = timed(g_fwd)
         torch.cuda.synchronize(dev)
         time.sleep(0.2)
     if world > 1:
         dist.barrier()
-    step_ms = [e0.elapsed_time(e1) for (e0, _, _, e1) in ev]
-    fwd_ms = [f0.elapsed_time(f1) for (_, f0, f1, _) in ev]
+    if B.device_status(att.tmap, stream) != 0:
+        raise RuntimeError("device error word set during the timed steps")
+    step_ms = [e0.elapsed_time(e1) for (e0, e1) in ev_step]
+    fwd_ms = [e0.elapsed_time(e1) for (e0, e1) in ev_fwd]
     total_ms = sum(step_ms)
     if world > 1:
         t = torch.tensor([total_ms], device=dev)
@@ -303,7 +321,8 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, "desc": W.WORKLOADS[args.workload], "B": Bsz, "Hq": Hq, "Hkv": Hkv,
                    "N": N, "d": d, "block_q": bq, "block_k": bk, "seed": prob.seed, "visible_pairs": pairs,
-                   "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}"},
+                   "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}",
+                   "launch": "each step replayed as a CUDA graph (map build + forward)"},
         "frac_of_peak": {"burst": value / burst, "sustained": value / sustained, "spec_2250": value / 2250.0,
                          "peaks": src},
         "fwd_only": {"ms": fwd_avg_ms, "tflops": achieved},
@@ -312,7 +331,7 @@ def main():
                      "frac": achieved / burst, "traffic": None, "peak_kind": f"{src} burst bf16 dense"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms": statistics.mean(e2e_ms)},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 4 * args.steps,  # per step: 3 tile-map kernels + 1 forward kernel
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline and world == 1:
