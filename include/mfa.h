@@ -181,6 +181,34 @@ mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v
                    const mfa_mask_desc* mask, const mfa_tensor* out, float* lse,
                    void* stream);
 
+/* Size of the device array mfa_fwd_noalloc keeps its tile map and work
+ * counters in: 16 MiB, held on every GPU where the library's kernels are
+ * loaded, until the process exits. */
+#define MFA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* The forward pass for callers that cannot allocate device memory: for
+ * example a plugin inside a host application that owns the GPU allocator and
+ * passes in only the tensors, or code that must not allocate at this point of
+ * its pipeline. The paper has no counterpart; this is a convenience of the
+ * library. It does what mfa_build_tile_map followed by mfa_fwd do, but the
+ * tile map (block_q x block_k, each 64 or 128) and the forward pass's work
+ * counters live in a fixed array of MFA_NOALLOC_SCRATCH_BYTES that the library
+ * itself holds in device memory; nothing is allocated by anyone. mask->map is
+ * ignored. q, k, v, out and lse are as for mfa_fwd.
+ * - A map larger than MFA_NOALLOC_SCRATCH_BYTES (mfa_tile_map_bytes) returns
+ *   MFA_ERR_UNSUPPORTED before anything is launched.
+ * - dev_err: optional DEVICE pointer to one uint32; after the pass it receives
+ *   the device error bits (MFA_DEVERR_*) by a device-to-device copy on
+ *   `stream`. NULL skips the copy.
+ * - The first call on each device looks up the array's device address with
+ *   that device current; make that first call before any stream capture.
+ * - Every call on a device shares the one array and leaves its contents in it
+ *   (each call clears and rebuilds what it uses). Calls that overlap on the
+ *   GPU race: order them (one stream, or events between streams). */
+mfa_status mfa_fwd_noalloc(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v,
+                           const mfa_mask_desc* mask, int32_t block_q, int32_t block_k,
+                           const mfa_tensor* out, float* lse, uint32_t* dev_err, void* stream);
+
 /* Synchronise `stream`, read the map's error word into *err_bits (if not
  * NULL) and return MFA_ERR_DEVICE when it is non-zero, MFA_OK otherwise. */
 mfa_status mfa_get_device_status(const mfa_tile_map* map, void* stream, uint32_t* err_bits);

@@ -23,7 +23,8 @@ MFA_BF16, MFA_F32 = 0, 1
 DEVERR_BOUNDS, DEVERR_SEL, DEVERR_TIMEOUT, DEVERR_MAP = 1, 2, 4, 8
 
 EXPORTS = ("mfa_abi_version", "mfa_status_string", "mfa_tile_map_bytes", "mfa_tile_map_init",
-           "mfa_build_tile_map", "mfa_fwd", "mfa_get_device_status")
+           "mfa_build_tile_map", "mfa_fwd", "mfa_fwd_noalloc", "mfa_get_device_status")
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class MfaTensor(ctypes.Structure):
@@ -78,6 +79,11 @@ def load(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.mfa_fwd.restype = ctypes.c_int
     lib.mfa_fwd.argtypes = [ctypes.POINTER(MfaTensor)] * 3 + [ctypes.POINTER(MfaMaskDesc), ctypes.POINTER(MfaTensor),
                                                               ctypes.c_void_p, ctypes.c_void_p]
+    lib.mfa_fwd_noalloc.restype = ctypes.c_int
+    lib.mfa_fwd_noalloc.argtypes = [ctypes.POINTER(MfaTensor)] * 3 + [ctypes.POINTER(MfaMaskDesc), ctypes.c_int32,
+                                                                      ctypes.c_int32, ctypes.POINTER(MfaTensor),
+                                                                      ctypes.c_void_p, ctypes.c_void_p,
+                                                                      ctypes.c_void_p]
     lib.mfa_get_device_status.restype = ctypes.c_int
     lib.mfa_get_device_status.argtypes = [ctypes.POINTER(MfaTileMap), ctypes.c_void_p,
                                           ctypes.POINTER(ctypes.c_uint32)]
@@ -190,6 +196,18 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: DeviceMask, tm
     qd, kd, vd, od = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
     _check("mfa_fwd", load().mfa_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(dmask.desc),
                                      ctypes.byref(od), lse.data_ptr(), _stream_ptr(stream)))
+
+
+def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: DeviceMask, block_q: int, block_k: int,
+                out: torch.Tensor, lse: torch.Tensor, dev_err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Forward pass with the tile map in the library's own device array (no allocation by anyone)."""
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor")
+    qd, kd, vd, od = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
+    err_ptr = None if dev_err is None else dev_err.data_ptr()
+    _check("mfa_fwd_noalloc", load().mfa_fwd_noalloc(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd),
+                                                     ctypes.byref(dmask.desc), block_q, block_k, ctypes.byref(od),
+                                                     lse.data_ptr(), err_ptr, _stream_ptr(stream)))
 
 
 def device_status(tmap: TileMap, stream=None) -> int:
