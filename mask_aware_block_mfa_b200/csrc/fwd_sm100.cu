@@ -363,7 +363,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // =================== MMA issuer ===================
-    if (lane == 0) {
+    // The whole warp runs this loop converged (waits are made warp-uniform)
+    // and the tcgen05 helpers issue from one elected lane.
+    {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kRows, BK, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kRows, D, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
@@ -373,9 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int it = 0; ok; ++it) {
         const int rs = it % kRing;
-        if (!(ok = mbar_wait(&sched_full[rs], (it / kRing) & 1, s_abort))) break;
+        if (!(ok = warp_all(mbar_wait(&sched_full[rs], (it / kRing) & 1, s_abort)))) break;
         const WorkItem info = ring[rs];
-        mbar_arrive(&sched_empty[rs]);
+        if (lane == 0) mbar_arrive(&sched_empty[rs]);
         if (info.w < 0) break;
         const Tile (&t)[2] = info.t;
         bool pending[2] = {false, false}, first_pv[2] = {true, true}, qready[2] = {false, false};
@@ -384,9 +386,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // O_t += P_t V for the tile's pending k-tile.
         auto issue_pv = [&](int s) -> bool {
-          if (!mbar_wait(&p_full[s], pcount[s] & 1, s_abort)) return false;
+          if (!warp_all(mbar_wait(&p_full[s], pcount[s] & 1, s_abort))) return false;
           ++pcount[s];
-          if (!mbar_wait(&v_full[pstage[s]], pphase[s], s_abort)) return false;
+          if (!warp_all(mbar_wait(&v_full[pstage[s]], pphase[s], s_abort))) return false;
           tc_fence_after();
           const uint32_t a_p = tmem + s * BK;
           const uint32_t d_o = tmem + 2 * BK + s * D;
@@ -414,14 +416,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (ok && m.next(kt, in[0], in[1])) {
           const int st = kv_it % S;
           const uint32_t ph = (kv_it / S) & 1;
-          if (!(ok = mbar_wait(&k_full[st], ph, s_abort))) break;
+          if (!(ok = warp_all(mbar_wait(&k_full[st], ph, s_abort)))) break;
           tc_fence_after();
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (pending[s] && !(ok = issue_pv(s))) break;
             if (in[s]) {
               if (!qready[s]) {
-                if (!(ok = mbar_wait(&q_full[s], quse[s] & 1, s_abort))) break;
+                if (!(ok = warp_all(mbar_wait(&q_full[s], quse[s] & 1, s_abort)))) break;
                 tc_fence_after();
                 qready[s] = true;
               }
@@ -442,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               pphase[s] = ph;
               if (++nS[s] == t[s].n) umma_commit(&q_empty[s]);  // last read of Q_s in this item
             } else {
-              mbar_arrive(&v_empty[st]);  // this tile does not read V at this k-tile
+              if (lane == 0) mbar_arrive(&v_empty[st]);  // this tile does not read V at this k-tile
             }
           }
           if (!ok) break;
