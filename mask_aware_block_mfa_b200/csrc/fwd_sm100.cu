@@ -528,6 +528,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           bnd = dst;
           ++n_bnd;
         }
+        // Column-wise mask words for this tile, computed before S is ready
+        // (the bounds are already staged) so that only BK / 32 words are live
+        // beside the scores. The warp's 32 lanes hold 32 consecutive queries
+        // from qbase. Lane j turns column (32c + j)'s two intervals into one
+        // word of masked rows (bit l = query qbase + l), then a 32x32 bit
+        // transpose across the warp gives every lane its own row's bits for
+        // those columns.
+        uint32_t mrow[BK / 32];
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c) mrow[c] = 0u;
+        if (bnd != nullptr) {
+          const int qbase = qi - lane;
+#pragma unroll
+          for (int c = 0; c < BK / 32; ++c) {
+            const int4 v = bnd[c * 32 + lane];
+            uint32_t w = rows_in_interval(v.x - qbase, v.y - qbase) | rows_in_interval(v.z - qbase, v.w - qbase);
+            mrow[c] = transpose32_warp(w, lane);
+          }
+        }
         if (!(ok = warp_all(mbar_wait(&s_full[slot], s_cnt & 1, s_abort)))) break;
         ++s_cnt;
         tc_fence_after();
@@ -544,18 +563,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (partial) {
           const int jb = kt * BK;
           if (mk.kind == MFA_MASK_COLWISE) {
-            // The warp's 32 lanes hold 32 consecutive queries from qbase. Lane j
-            // turns column (32c + j)'s two intervals into one word of masked
-            // rows (bit l = query qbase + l), then a 32x32 bit transpose across
-            // the warp gives every lane its own row's bits for those columns.
-            const int qbase = qi - lane;
-            uint32_t mrow[BK / 32];
-#pragma unroll
-            for (int c = 0; c < BK / 32; ++c) {
-              const int4 v = bnd[c * 32 + lane];
-              uint32_t w = rows_in_interval(v.x - qbase, v.y - qbase) | rows_in_interval(v.z - qbase, v.w - qbase);
-              mrow[c] = transpose32_warp(w, lane);
-            }
 #pragma unroll
             for (int jj = 0; jj < BK; ++jj)
               if ((mrow[jj >> 5] >> (jj & 31)) & 1u) s[jj] = -INFINITY;
@@ -583,25 +590,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool need = mx_s > m_run + kRescaleThreshold;
         const float m_new = need ? mx_s : m_run;
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        float sum = 0.f;
+        // P = 2^(s * scale - m) as bf16 over S, 32 columns at a time so that
+        // only 16 packed registers are live beside s[]. S_t(i) being complete
+        // implies P_t(i-1).V is complete (MMAs finish in issue order), so S and
+        // O of this slot are free here. Four partial sums keep the FADD chain
+        // short.
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int jj = 0; jj < BK; ++jj) {
-          const float e = ex2_approx(fmaf(s[jj], p.scale_log2, -m_use));
-          s[jj] = e;
-          sum += e;
+        for (int c = 0; c < BK / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float e0 = ex2_approx(fmaf(s[c * 32 + 2 * u], p.scale_log2, -m_use));
+            const float e1 = ex2_approx(fmaf(s[c * 32 + 2 * u + 1], p.scale_log2, -m_use));
+            sum4[u & 3] += e0 + e1;
+            pk[u] = pack_bf16x2(e0, e1);
+          }
+          tmem_st_32x32b_x16(tmem_s + lane_off + c * 16, pk);
         }
+        const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
         const float alpha = need ? ex2_approx(m_run - m_use) : 1.f;
         l_run = l_run * alpha + sum;
         m_run = m_new;
-        // P (bf16) over S. S_t(i) being complete implies P_t(i-1).V is complete
-        // (MMAs finish in issue order), so S and O of this slot are free here.
-#pragma unroll
-        for (int c = 0; c < BK / 64; ++c) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int u = 0; u < 32; ++u) pk[u] = pack_bf16x2(s[c * 64 + 2 * u], s[c * 64 + 2 * u + 1]);
-          tmem_st_32x32b_x32(tmem_s + lane_off + c * 32, pk);
-        }
         if (i > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
