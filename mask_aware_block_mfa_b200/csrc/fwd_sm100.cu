@@ -69,6 +69,7 @@ struct FwdParams {
   const int32_t* order;
   __nv_bfloat16* out;
   int64_t os0, os1, os2;
+  int32_t out_v8;  // 1: out and its strides are 32-byte aligned (256-bit stores)
   float* lse;
   uint32_t* err;
   uint32_t* sched;  // [0] next work item, [1] CTAs finished (map scratch words)
@@ -642,6 +643,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool store = qi < p.Nq;
       __nv_bfloat16* orow = p.out + static_cast<int64_t>(T.b) * p.os0 + static_cast<int64_t>(head) * p.os1 +
                             static_cast<int64_t>(qi) * p.os2;
+      // Each thread writes its own row. With 32-byte aligned rows a store
+      // covers whole 32-byte sectors; 16-byte stores would write every sector
+      // in two halves from two instructions.
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -650,14 +654,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
         }
         if (store) {
+          uint32_t w[16];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            uint4 v;
-            v.x = has ? pack_bf16x2(__uint_as_float(o[8 * g + 0]) * inv, __uint_as_float(o[8 * g + 1]) * inv) : 0u;
-            v.y = has ? pack_bf16x2(__uint_as_float(o[8 * g + 2]) * inv, __uint_as_float(o[8 * g + 3]) * inv) : 0u;
-            v.z = has ? pack_bf16x2(__uint_as_float(o[8 * g + 4]) * inv, __uint_as_float(o[8 * g + 5]) * inv) : 0u;
-            v.w = has ? pack_bf16x2(__uint_as_float(o[8 * g + 6]) * inv, __uint_as_float(o[8 * g + 7]) * inv) : 0u;
-            reinterpret_cast<uint4*>(orow)[c * 4 + g] = v;
+          for (int u = 0; u < 16; ++u)
+            w[u] = has ? pack_bf16x2(__uint_as_float(o[2 * u]) * inv, __uint_as_float(o[2 * u + 1]) * inv) : 0u;
+          if (p.out_v8) {
+            st_global_v8(orow + c * 32, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+            st_global_v8(orow + c * 32 + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+          } else {
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              reinterpret_cast<uint4*>(orow)[c * 4 + g] = make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
           }
         }
       }
@@ -812,6 +819,10 @@ extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   p.cls = map->tile_class; p.list = map->tile_list; p.count = map->tile_count; p.order = map->order;
   p.out = static_cast<__nv_bfloat16*>(out->data);
   p.os0 = out->stride[0]; p.os1 = out->stride[1]; p.os2 = out->stride[2];
+  p.out_v8 = (reinterpret_cast<uintptr_t>(out->data) % 32 == 0 && out->stride[0] % 16 == 0 &&
+              out->stride[1] % 16 == 0 && out->stride[2] % 16 == 0)
+                 ? 1
+                 : 0;
   p.lse = lse;
   p.err = map->err;
   p.sched = map->err + 1;

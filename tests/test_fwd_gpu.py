@@ -115,6 +115,31 @@ def test_fwd_all_rows_masked():
     assert torch.isneginf(lse).all() and (out == 0).all()
 
 
+@pytest.mark.parametrize("layout", ["offset16", "bnhd"])
+def test_fwd_output_layouts(layout):
+    """The epilogue writes 32-byte pieces of a row when out and its strides are
+    32-byte aligned and 16-byte pieces otherwise: an out that starts 16 bytes
+    past an aligned address takes the second path, a [B, N, H, D] view (rows of
+    one head H * D apart) the first one with a non-contiguous row stride."""
+    mask = W.make_mask("doc8k", N=1024)
+    prob = small_problem(mask, 4, 2, 128, seed=12)
+    att = B.Attention(prob.mask, 64, 128)
+    att.build()
+    q, k, v = (t.to("cuda") for t in (prob.q, prob.k, prob.v))
+    Bn, Hq, Nq, d = q.shape
+    if layout == "offset16":
+        buf = torch.zeros(q.numel() + 8, dtype=torch.bfloat16, device="cuda")
+        out = buf[8:].view(Bn, Hq, Nq, d)
+        assert out.data_ptr() % 32 == 16
+    else:
+        out = torch.zeros(Bn, Nq, Hq, d, dtype=torch.bfloat16, device="cuda").permute(0, 2, 1, 3)
+    lse = torch.empty(Bn, Hq, Nq, dtype=torch.float32, device="cuda")
+    att(q, k, v, out, lse)
+    assert B.device_status(att.tmap) == 0
+    ref_out, ref_lse = oracle_rows(prob, None)
+    compare_attention(out.float().cpu(), lse.cpu(), ref_out, ref_lse)
+
+
 def test_fwd_deterministic():
     prob = small_problem(W.make_mask("doc8k", N=1024), 4, 2, 128, seed=6)
     a, la, _, _ = run_gpu(prob, 64, 128)
