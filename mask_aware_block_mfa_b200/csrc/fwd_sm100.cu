@@ -529,23 +529,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           bnd = dst;
           ++n_bnd;
         }
-        // Column-wise mask words for this tile, computed before S is ready
-        // (the bounds are already staged) so that only BK / 32 words are live
-        // beside the scores. The warp's 32 lanes hold 32 consecutive queries
-        // from qbase. Lane j turns column (32c + j)'s two intervals into one
-        // word of masked rows (bit l = query qbase + l), then a 32x32 bit
-        // transpose across the warp gives every lane its own row's bits for
-        // those columns.
+        // Masked columns of this row in a PARTIAL tile, as BK / 32 words (bit
+        // j of word c = column 32c + j), built before S is ready so that one
+        // short loop applies every mask kind and only these words are live
+        // beside the scores.
+        //   column-wise: the warp's 32 lanes hold 32 consecutive queries from
+        //     qbase; lane j turns column (32c + j)'s two intervals into a word
+        //     of masked rows (bit l = query qbase + l), and a 32x32 bit
+        //     transpose across the warp gives each lane its own row's columns
+        //     (columns past Nk are staged as masked for every row);
+        //   band: the visible columns form one interval per row;
+        //   block selection: the causal interval, cleared in the 64-column
+        //     halves that the tile's class byte does not select.
         uint32_t mrow[BK / 32];
 #pragma unroll
         for (int c = 0; c < BK / 32; ++c) mrow[c] = 0u;
-        if (bnd != nullptr) {
-          const int qbase = qi - lane;
+        if (partial) {
+          const int jb = kt * BK;
+          if (bnd != nullptr) {
+            const int qbase = qi - lane;
 #pragma unroll
-          for (int c = 0; c < BK / 32; ++c) {
-            const int4 v = bnd[c * 32 + lane];
-            uint32_t w = rows_in_interval(v.x - qbase, v.y - qbase) | rows_in_interval(v.z - qbase, v.w - qbase);
-            mrow[c] = transpose32_warp(w, lane);
+            for (int c = 0; c < BK / 32; ++c) {
+              const int4 v = bnd[c * 32 + lane];
+              const uint32_t w =
+                  rows_in_interval(v.x - qbase, v.y - qbase) | rows_in_interval(v.z - qbase, v.w - qbase);
+              mrow[c] = transpose32_warp(w, lane);
+            }
+          } else if (mk.kind == MFA_MASK_BAND) {
+            const int lo = qi - mk.pre - jb;                  // first visible column of the tile
+            const int hi = min(qi + mk.nxt - jb + 1, p.Nk - jb);  // one past the last one
+#pragma unroll
+            for (int c = 0; c < BK / 32; ++c) mrow[c] = ~rows_in_interval(lo - 32 * c, hi - 32 * c);
+          } else {
+            const int qsl = (GP == 2) ? 0 : (r >> 6);
+            const int hi = min(qi - jb + 1, p.Nk - jb);
+#pragma unroll
+            for (int c = 0; c < BK / 32; ++c) {
+              const bool sel = (cb >> (4 + 2 * qsl + (c >> 1))) & 1u;
+              mrow[c] = sel ? ~rows_in_interval(-32 * c, hi - 32 * c) : ~0u;
+            }
           }
         }
         if (!(ok = warp_all(mbar_wait(&s_full[slot], s_cnt & 1, s_abort)))) break;
@@ -562,27 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int jj = 0; jj < BK; ++jj) s[jj] = __uint_as_float(sv[jj >> 5][jj & 31]);
         }
         if (partial) {
-          const int jb = kt * BK;
-          if (mk.kind == MFA_MASK_COLWISE) {
 #pragma unroll
-            for (int jj = 0; jj < BK; ++jj)
-              if ((mrow[jj >> 5] >> (jj & 31)) & 1u) s[jj] = -INFINITY;
-          } else if (mk.kind == MFA_MASK_BAND) {
-#pragma unroll
-            for (int jj = 0; jj < BK; ++jj) {
-              const int dj = jb + jj - qi;
-              const bool vis = (jb + jj < p.Nk) && dj >= -mk.pre && dj <= mk.nxt;
-              if (!vis) s[jj] = -INFINITY;
-            }
-          } else {
-            const int qsl = (GP == 2) ? 0 : (r >> 6);
-#pragma unroll
-            for (int jj = 0; jj < BK; ++jj) {
-              const int ksl = jj >> 6;
-              const bool vis = (jb + jj < p.Nk) && (jb + jj <= qi) && ((cb >> (4 + 2 * qsl + ksl)) & 1u);
-              if (!vis) s[jj] = -INFINITY;
-            }
-          }
+          for (int jj = 0; jj < BK; ++jj)
+            if ((mrow[jj >> 5] >> (jj & 31)) & 1u) s[jj] = -INFINITY;
         }
         float mx = -INFINITY;
 #pragma unroll
