@@ -374,6 +374,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pcount[2] = {0, 0};
       int quse[2] = {0, 0};
       bool ok = true;
+      // The P.V of a tile's last k-tile is not issued at the end of its work
+      // item but carried into the next item, where it goes out just before that
+      // slot's first S like any pending P.V. The MMA warp thus reads the next
+      // ring entry and sets up the next item while the softmax still works on
+      // the last P, and the next S follows the carried P.V at once. Each
+      // pending P.V records its V stage and whether it is the first (O is
+      // overwritten) or last (o_done is committed) P.V of its item.
+      // Per slot s, bits of `pv`: 1 << s pending, 4 << s first, 16 << s last;
+      // pkv[s] = the k-tile counter of the pending P.V (stage and phase of V).
+      uint32_t pv = 0;
+      uint32_t pkv[2] = {0, 0};
+
+      // O_t += P_t V for the tile's pending k-tile.
+      auto issue_pv = [&](int s) -> bool {
+        if (!warp_all(mbar_wait(&p_full[s], pcount[s] & 1, s_abort))) return false;
+        ++pcount[s];
+        const uint32_t vst = pkv[s] % S;
+        if (!warp_all(mbar_wait(&v_full[vst], (pkv[s] / S) & 1, s_abort))) return false;
+        tc_fence_after();
+        const uint32_t a_p = tmem + s * BK;
+        const uint32_t d_o = tmem + 2 * BK + s * D;
+        // Descriptor start addresses are in 16-byte units in the low bits, so
+        // advancing by a byte offset adds offset >> 4 to the descriptor.
+        // The MMAs are issued fully unrolled: a rolled issue loop costs about
+        // twice the MMA's own 64 cycles per instruction.
+        const uint64_t vd = sdesc_sw128(v_addr + vst * C::kKVBytes, BK * 128, 1024);
+        umma_ts(d_o, a_p, vd, idesc_pv, (pv & (4u << s)) ? 0u : 1u);
+#pragma unroll
+        for (int kk = 1; kk < BK / 16; ++kk)
+          umma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * (16 * 128 / 16)), idesc_pv, 1u);
+        // The next S of this slot is issued after this P.V, so its s_full
+        // commit also covers this MMA; o_done is needed only after the item's
+        // last P.V.
+        if (pv & (16u << s)) umma_commit(&o_done[s]);
+        umma_commit(&v_empty[vst]);
+        pv &= ~(21u << s);
+        return true;
+      };
+
       for (int it = 0; ok; ++it) {
         const int rs = it % kRing;
         if (!(ok = warp_all(mbar_wait(&sched_full[rs], (it / kRing) & 1, s_abort)))) break;
@@ -381,47 +420,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sched_empty[rs]);
         if (info.w < 0) break;
         const Tile (&t)[2] = info.t;
-        bool pending[2] = {false, false}, first_pv[2] = {true, true}, qready[2] = {false, false};
-        int pstage[2] = {0, 0}, nS[2] = {0, 0}, nPV[2] = {0, 0};
-        uint32_t pphase[2] = {0, 0};
-
-        // O_t += P_t V for the tile's pending k-tile.
-        auto issue_pv = [&](int s) -> bool {
-          if (!warp_all(mbar_wait(&p_full[s], pcount[s] & 1, s_abort))) return false;
-          ++pcount[s];
-          if (!warp_all(mbar_wait(&v_full[pstage[s]], pphase[s], s_abort))) return false;
-          tc_fence_after();
-          const uint32_t a_p = tmem + s * BK;
-          const uint32_t d_o = tmem + 2 * BK + s * D;
-          // Descriptor start addresses are in 16-byte units in the low bits, so
-          // advancing by a byte offset adds offset >> 4 to the descriptor.
-          // The MMAs are issued fully unrolled: a rolled issue loop costs about
-          // twice the MMA's own 64 cycles per instruction.
-          const uint64_t vd = sdesc_sw128(v_addr + pstage[s] * C::kKVBytes, BK * 128, 1024);
-          umma_ts(d_o, a_p, vd, idesc_pv, first_pv[s] ? 0u : 1u);
-#pragma unroll
-          for (int kk = 1; kk < BK / 16; ++kk)
-            umma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * (16 * 128 / 16)), idesc_pv, 1u);
-          // S_t of the next k-tile is issued after this P.V, so its s_full commit
-          // also covers this MMA; o_done is needed only after the tile's last P.V.
-          if (++nPV[s] == t[s].n) umma_commit(&o_done[s]);
-          umma_commit(&v_empty[pstage[s]]);
-          first_pv[s] = false;
-          pending[s] = false;
-          return true;
-        };
+        bool qready[2] = {false, false};
+        int nS[2] = {0, 0};
 
         Merge m = make_merge(p, t);
         int kt;
         bool in[2];
+        bool first_kt = true;
         while (ok && m.next(kt, in[0], in[1])) {
           const int st = kv_it % S;
           const uint32_t ph = (kv_it / S) & 1;
+          // At an item's first k-tile the pending P.V are the previous item's
+          // last ones: they need no K, and the item's first K tile may still be
+          // loading, so slot 0's goes out before the K wait and slot 1's too if
+          // K has not landed. Later k-tiles keep the order K, PV_0, S_0, PV_1,
+          // S_1.
+          if (first_kt) {
+            first_kt = false;
+            if ((pv & 1u) && !(ok = issue_pv(0))) break;
+            if ((pv & 2u) && !warp_all(mbar_try_wait(&k_full[st], ph)) && !(ok = issue_pv(1))) break;
+          }
           if (!(ok = warp_all(mbar_wait(&k_full[st], ph, s_abort)))) break;
           tc_fence_after();
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
-            if (pending[s] && !(ok = issue_pv(s))) break;
+            if ((pv & (1u << s)) && !(ok = issue_pv(s))) break;
             if (in[s]) {
               if (!qready[s]) {
                 if (!(ok = warp_all(mbar_wait(&q_full[s], quse[s] & 1, s_abort)))) break;
@@ -440,10 +463,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_ss(tmem + s * BK, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
               }
               umma_commit(&s_full[s]);
-              pending[s] = true;
-              pstage[s] = st;
-              pphase[s] = ph;
-              if (++nS[s] == t[s].n) umma_commit(&q_empty[s]);  // last read of Q_s in this item
+              pkv[s] = kv_it;
+              const bool last = ++nS[s] == t[s].n;
+              pv |= (1u << s) | (nS[s] == 1 ? (4u << s) : 0u) | (last ? (16u << s) : 0u);
+              if (last) umma_commit(&q_empty[s]);  // last read of Q_s in this item
             } else {
               if (lane == 0) mbar_arrive(&v_empty[st]);  // this tile does not read V at this k-tile
             }
@@ -454,11 +477,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int s = 0; s < 2; ++s)
-          if (ok && pending[s]) ok = issue_pv(s);
-#pragma unroll
-        for (int s = 0; s < 2; ++s)
           if (t[s].n > 0) ++quse[s];
       }
+      // The P.V still pending when the work runs out.
+#pragma unroll
+      for (int s = 0; s < 2; ++s)
+        if (ok && (pv & (1u << s))) ok = issue_pv(s);
       if (!ok) *s_abort = 1;
       // Wait for every MMA issued here before TMEM can be released.
       umma_commit(drain);
@@ -588,9 +612,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int jj = 0; jj < BK; ++jj)
             if ((mrow[jj >> 5] >> (jj & 31)) & 1u) s[jj] = -INFINITY;
         }
-        float mx = -INFINITY;
+        // Row max with 3-input max instructions over four independent chains.
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int jj = 0; jj < BK; ++jj) mx = fmaxf(mx, s[jj]);
+        for (int jj = 0; jj < BK; jj += 8)
+#pragma unroll
+          for (int a = 0; a < 4; ++a) mx4[a] = fmax3(mx4[a], s[jj + 2 * a], s[jj + 2 * a + 1]);
+        const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
         const float mx_s = mx * p.scale_log2;
         const bool need = mx_s > m_run + kRescaleThreshold;
         const float m_new = need ? mx_s : m_run;
@@ -618,7 +646,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run = l_run * alpha + sum;
         m_run = m_new;
         if (i > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
+          // Rare (the running max grew by more than the threshold): kept
+          // rolled to save instruction-cache space for the hot path.
+#pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
             tmem_ld_32x32b_x32(tmem_o + lane_off + c * 32, o);
@@ -626,6 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
             tmem_st_32x32b_x32(tmem_o + lane_off + c * 32, o);
+            tmem_st_wait();
           }
         }
         tmem_st_wait();
@@ -649,8 +680,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             static_cast<int64_t>(qi) * p.os2;
       // Each thread writes its own row. With 32-byte aligned rows a store
       // covers whole 32-byte sectors; 16-byte stores would write every sector
-      // in two halves from two instructions.
-#pragma unroll
+      // in two halves from two instructions. The chunk loop stays rolled: it
+      // runs once per item.
+#pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         if (n > 0) {

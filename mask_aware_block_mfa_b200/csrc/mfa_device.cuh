@@ -31,25 +31,72 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA/ALU pipes instead of the MUFU unit. Cody and Waite's range
-// reduction: x = j + f with j = round(x) (adding 1.5 * 2^23 leaves round(x) in
-// the low mantissa bits) and f in [-1/2, 1/2]; 2^f from the degree-3 polynomial
-// of minimum relative error on [-1/2, 1/2] (Remez exchange, coefficients from
-// csrc/exp2_poly_fit.py, max relative error 7.5e-5 in float32); 2^j is added
-// to the exponent field. Exactly 0 below -125, so masked (-inf) scores give 0.
+// Packed pairs of float32 (low half = first element) for the sm_100 f32x2
+// instructions: one issue slot operates on two values.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a packed pair on the FMA/ALU pipes instead of the MUFU unit.
+// Cody and Waite's range reduction: x = j + f with j = round(x) (adding
+// 1.5 * 2^23 leaves round(x) in the low mantissa bits) and f in [-1/2, 1/2];
+// 2^f from the degree-3 polynomial of minimum relative error on [-1/2, 1/2]
+// (Remez exchange, coefficients from csrc/exp2_poly_fit.py, max relative error
+// 7.5e-5 in float32); 2^j is added to the exponent field. Inputs below -125
+// (masked scores are -inf) are clamped there and give about 2^-125, not 0:
+// the caller must treat a row with no visible key separately.
 constexpr float kExp2C0 = 0x1.fff692p-1f;
 constexpr float kExp2C1 = 0x1.62f31ap-1f;
 constexpr float kExp2C2 = 0x1.f0de1ap-3f;
 constexpr float kExp2C3 = 0x1.c3f76p-5f;
 
-__device__ __forceinline__ float exp2_poly(float x) {
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = f2_add(xc, f2_pack(kShift, kShift));
+  const uint64_t j = f2_add(t, f2_pack(-kShift, -kShift));
+  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), xc);
+  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
+// The same 2^x for one value with the coefficients as instruction immediates
+// (no registers held across a loop); same clamp at -125.
+__device__ __forceinline__ float exp2_poly1(float x) {
   const float xc = fmaxf(x, -125.f);
   const float t = __fadd_rn(xc, 12582912.f);
-  const float j = __fsub_rn(t, 12582912.f);
+  const float j = __fadd_rn(t, -12582912.f);
   const float f = __fsub_rn(xc, j);
   const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-  const uint32_t bits = __float_as_uint(p) + (__float_as_uint(t) << 23);
-  return x < -125.f ? 0.f : __uint_as_float(bits);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

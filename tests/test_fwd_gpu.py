@@ -140,6 +140,30 @@ def test_fwd_output_layouts(layout):
     compare_attention(out.float().cpu(), lse.cpu(), ref_out, ref_lse)
 
 
+def test_fwd_rows_without_keys_inside_visible_tiles():
+    """Causal mask in which queries 100..109 see no key at all while the other
+    rows of their tiles do. Those rows run through PARTIAL and FULL tiles with a
+    running max of -inf; they must still give out = 0 and lse = -inf (their
+    exponentials from the FMA-pipe exp2 are about 2^-125, not 0, so the kernel
+    has to zero their row sum), and the rows around them must be unaffected."""
+    N = 600
+    j = np.arange(N, dtype=np.int32)
+    uts = np.zeros((1, 1, N), np.int32)
+    ute = j.reshape(1, 1, N).copy()                    # causal: rows < j masked
+    lts = np.maximum(100, j).astype(np.int32).reshape(1, 1, N)
+    lte = np.full((1, 1, N), 110, np.int32)
+    lte = np.where(j.reshape(1, 1, N) < 110, lte, lts)  # rows [max(100, j), 110) masked
+    mask = W.MaskDesc(W.MASK_COLWISE, 1, 1, N, N, lts, lte.astype(np.int32), uts, ute, name="holes")
+    prob = small_problem(mask, 4, 2, 128, seed=21)
+    for bq, bk in ((64, 128), (128, 64)):
+        out, lse, arrays, err = run_gpu(prob, bq, bk)
+        assert err == 0
+        compare_map(arrays, prob.mask, bq, bk)
+        ref_out, ref_lse = oracle_rows(prob, None)
+        assert np.isneginf(ref_lse[:, :, 100:110]).all() and np.isfinite(ref_lse[:, :, 110:]).all()
+        compare_attention(out, lse, ref_out, ref_lse)
+
+
 def test_fwd_deterministic():
     prob = small_problem(W.make_mask("doc8k", N=1024), 4, 2, 128, seed=6)
     a, la, _, _ = run_gpu(prob, 64, 128)
