@@ -16,6 +16,7 @@ the value is the sum of all ranks' work over the slowest rank's time.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -42,6 +43,30 @@ BLOCKS = {  # launch configuration per workload: (block_q, block_k)
     "blocksel32k": (64, 64),
 }
 METRIC = "effective TFLOP/s (visible pairs only) and % of B200 bf16 tensor peak"
+
+# DRAM bytes (read + write) of one forward launch, from one ncu capture of
+# the forward kernel on that workload (the summaries under profiles/ give the
+# command). Each entry holds the digest of the kernel sources it was taken
+# on; a changed kernel reports traffic as null until it is captured again.
+KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/fwd_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh")
+NCU_TRAFFIC = {
+    "doc8k": (135_357_184, "77a27b2753d0c19d"),
+    "doc32k": (1_040_363_008, "77a27b2753d0c19d"),
+}
+
+
+def kernel_digest() -> str:
+    h = hashlib.sha256()
+    root = os.path.dirname(os.path.abspath(__file__))
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(root, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    entry = NCU_TRAFFIC.get(workload)
+    return entry[0] if entry and entry[1] == kernel_digest() else None
 
 
 def peaks():
@@ -328,7 +353,8 @@ def main():
         "fwd_only": {"ms": fwd_avg_ms, "tflops": achieved},
         "map_ms": ms_per_step - fwd_avg_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
-                     "frac": achieved / burst, "traffic": None, "peak_kind": f"{src} burst bf16 dense"},
+                     "frac": achieved / burst, "traffic": ncu_traffic(args.workload),
+                     "peak_kind": f"{src} burst bf16 dense"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms": statistics.mean(e2e_ms)},
         "gpu_launches": 4 * args.steps,  # per step: 3 tile-map kernels + 1 forward kernel

@@ -21,3 +21,13 @@ def test_full_size_counts_are_plausible():
     assert 0.02 < frac < 0.2
     m = W.make_mask("band16k")
     assert bench.visible_pairs(m) == 2 * sum(min(i, 2048) + 1 for i in range(16384))
+
+
+def test_ncu_traffic_follows_the_kernel_digest():
+    import bench
+    digest = bench.kernel_digest()
+    assert len(digest) == 16 and int(digest, 16) >= 0
+    assert bench.ncu_traffic("no-such-workload") is None
+    for name, (nbytes, dig) in bench.NCU_TRAFFIC.items():
+        assert nbytes > 0 and len(dig) == 16
+        assert bench.ncu_traffic(name) == (nbytes if dig == digest else None)
