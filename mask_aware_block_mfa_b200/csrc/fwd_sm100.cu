@@ -88,14 +88,18 @@ struct Cfg {
   static constexpr int kV = kK + kStages * kKVBytes;
   static constexpr int kBar = kV + kStages * kKVBytes;
   // q_full[2] q_empty[2] k_full[S] k_empty[S] v_full[S] v_empty[S] s_full[2] p_full[2]
-  // o_done[2] bnd[2][2] drain sched_full[kRing] sched_empty[kRing]
-  static constexpr int kNumBars = 4 + 4 * kStages + 6 + 4 + 1 + 2 * kRing;
+  // s_full[2][2] p_full[2][2] o_done[2] pv_done[2] bnd[2][2] drain sched_full[kRing] sched_empty[kRing]
+  static constexpr int kNumBars = 4 + 4 * kStages + 12 + 4 + 1 + 2 * kRing;
   static constexpr int kBounds = kBar + ((kNumBars * 8 + 15) / 16) * 16;  // int4 [2 tiles][2 slots][BK]
   static constexpr int kRingOff = kBounds + 4 * BK * 16;                 // WorkItem [kRing]
   static constexpr int kMisc = kRingOff + kRing * 128;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
-  static constexpr int kTmemCols = (2 * BK + 2 * D) <= 256 ? 256 : 512;
+  // S buffers per tile in TMEM: two when BK = 64 (4 x 64 S + 2 x 128 O columns
+  // fit in 512), so S_t(u+1) is computed while the softmax works on S_t(u).
+  static constexpr int kSBufs = BK == 64 ? 2 : 1;
+  static constexpr int kTmemCols = (2 * kSBufs * BK + 2 * D) <= 256 ? 256 : 512;
+  static constexpr int kOCol = 2 * kSBufs * BK;  // first O column
 };
 
 struct Tile {
@@ -234,9 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_full = k_empty + S;
   uint64_t* v_empty = v_full + S;
   uint64_t* s_full = v_empty + S;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* bnd_full = o_done + 2;  // [2 tiles][2 slots]
+  uint64_t* p_full = s_full + 4;  // [tile][S buffer], like s_full
+  uint64_t* o_done = p_full + 4;
+  uint64_t* pv_done = o_done + 2;  // one phase per P.V of the tile
+  uint64_t* bnd_full = pv_done + 2;  // [2 tiles][2 slots]
   uint64_t* drain = bnd_full + 4;
   uint64_t* sched_full = drain + 1;
   uint64_t* sched_empty = sched_full + kRing;
@@ -253,9 +258,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&q_full[t], 1);
       mbar_init(&q_empty[t], 1);
-      mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], kRows);
+      mbar_init(&s_full[2 * t], 1);
+      mbar_init(&s_full[2 * t + 1], 1);
+      mbar_init(&p_full[2 * t], kRows);
+      mbar_init(&p_full[2 * t + 1], kRows);
       mbar_init(&o_done[t], 1);
+      mbar_init(&pv_done[t], 1);
       mbar_init(&bnd_full[2 * t], kRows);
       mbar_init(&bnd_full[2 * t + 1], kRows);
     }
@@ -371,7 +379,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kRows, D, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
       uint32_t kv_it = 0;
-      uint32_t pcount[2] = {0, 0};
+      // nsq[t] counts the S_t issued so far; S number k of a tile uses S buffer
+      // k % kSBufs and the phase (k / kSBufs) & 1 of that buffer's s_full and
+      // p_full. psq[t] is the S number of the tile's pending P.V.
+      uint32_t nsq[2] = {0, 0}, psq[2] = {0, 0};
       int quse[2] = {0, 0};
       bool ok = true;
       // The P.V of a tile's last k-tile is not issued at the end of its work
@@ -388,13 +399,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // O_t += P_t V for the tile's pending k-tile.
       auto issue_pv = [&](int s) -> bool {
-        if (!warp_all(mbar_wait(&p_full[s], pcount[s] & 1, s_abort))) return false;
-        ++pcount[s];
+        const uint32_t sb = psq[s] % C::kSBufs;
+        if (!warp_all(mbar_wait(&p_full[2 * s + sb], (psq[s] / C::kSBufs) & 1, s_abort))) return false;
         const uint32_t vst = pkv[s] % S;
         if (!warp_all(mbar_wait(&v_full[vst], (pkv[s] / S) & 1, s_abort))) return false;
         tc_fence_after();
-        const uint32_t a_p = tmem + s * BK;
-        const uint32_t d_o = tmem + 2 * BK + s * D;
+        const uint32_t a_p = tmem + (s * C::kSBufs + sb) * BK;
+        const uint32_t d_o = tmem + C::kOCol + s * D;
         // Descriptor start addresses are in 16-byte units in the low bits, so
         // advancing by a byte offset adds offset >> 4 to the descriptor.
         // The MMAs are issued fully unrolled: a rolled issue loop costs about
@@ -404,10 +415,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 1; kk < BK / 16; ++kk)
           umma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * (16 * 128 / 16)), idesc_pv, 1u);
-        // The next S of this slot is issued after this P.V, so its s_full
-        // commit also covers this MMA; o_done is needed only after the item's
-        // last P.V.
+        // With one S buffer the next S of this slot is issued after this P.V,
+        // so its s_full commit also covers this MMA; o_done is needed only
+        // after the item's last P.V.
         if (pv & (16u << s)) umma_commit(&o_done[s]);
+        umma_commit(&pv_done[s]);
         umma_commit(&v_empty[vst]);
         pv &= ~(21u << s);
         return true;
@@ -421,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (info.w < 0) break;
         const Tile (&t)[2] = info.t;
         bool qready[2] = {false, false};
-        int nS[2] = {0, 0};
+        uint32_t nS[2] = {0, 0};
 
         Merge m = make_merge(p, t);
         int kt;
@@ -434,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // last ones: they need no K, and the item's first K tile may still be
           // loading, so slot 0's goes out before the K wait and slot 1's too if
           // K has not landed. Later k-tiles keep the order K, PV_0, S_0, PV_1,
-          // S_1.
+          // S_1 (one S buffer per tile) or K, S_0, S_1, PV_0, PV_1 (two).
           if (first_kt) {
             first_kt = false;
             if ((pv & 1u) && !(ok = issue_pv(0))) break;
@@ -442,33 +454,71 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!(ok = warp_all(mbar_wait(&k_full[st], ph, s_abort)))) break;
           tc_fence_after();
+          // S_s = Q_s K^T for k-tile st; returns the pending-P.V flags it adds.
+          auto issue_s = [&](int s) -> uint32_t {
+            const uint32_t sb = nsq[s] % C::kSBufs;
+            const uint64_t qd = sdesc_sw128(q_addr + s * C::kQBytes, 16, 1024);
+            const uint64_t kd = sdesc_sw128(k_addr + st * C::kKVBytes, 16, 1024);
 #pragma unroll
-          for (int s = 0; s < 2; ++s) {
-            if ((pv & (1u << s)) && !(ok = issue_pv(s))) break;
-            if (in[s]) {
-              if (!qready[s]) {
-                if (!(ok = warp_all(mbar_wait(&q_full[s], quse[s] & 1, s_abort)))) break;
-                tc_fence_after();
-                qready[s] = true;
-              }
-              const uint64_t qd = sdesc_sw128(q_addr + s * C::kQBytes, 16, 1024);
-              const uint64_t kd = sdesc_sw128(k_addr + st * C::kKVBytes, 16, 1024);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              // K step of 16 bf16 = 32 bytes inside the 128-byte row; every 4
+              // steps move to the next 64-column chunk of the tile.
+              const uint32_t off = (kk & 3) * 32;
+              const uint64_t a = qd + static_cast<uint64_t>(((kk >> 2) * (kRows * 128) + off) >> 4);
+              const uint64_t bd = kd + static_cast<uint64_t>(((kk >> 2) * (BK * 128) + off) >> 4);
+              umma_ss(tmem + (s * C::kSBufs + sb) * BK, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[2 * s + sb]);
+            ++nsq[s];
+            const bool last = ++nS[s] == t[s].n;
+            if (last) umma_commit(&q_empty[s]);  // last read of Q_s in this item
+            return (1u << s) | (nS[s] == 1 ? (4u << s) : 0u) | (last ? (16u << s) : 0u);
+          };
+          auto q_ready = [&](int s) -> bool {
+            if (qready[s]) return true;
+            if (!warp_all(mbar_wait(&q_full[s], quse[s] & 1, s_abort))) return false;
+            tc_fence_after();
+            qready[s] = true;
+            return true;
+          };
+          if constexpr (C::kSBufs == 2) {
+            // Two S buffers per tile: both S of this k-tile go out first (into
+            // the buffers the pending P.V do not read), then the pending P.V.
+            uint32_t added = 0;
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                // K step of 16 bf16 = 32 bytes inside the 128-byte row; every 4
-                // steps move to the next 64-column chunk of the tile.
-                const uint32_t off = (kk & 3) * 32;
-                const uint64_t a = qd + static_cast<uint64_t>(((kk >> 2) * (kRows * 128) + off) >> 4);
-                const uint64_t bd = kd + static_cast<uint64_t>(((kk >> 2) * (BK * 128) + off) >> 4);
-                umma_ss(tmem + s * BK, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+            for (int s = 0; s < 2; ++s) {
+              if (in[s]) {
+                if (!(ok = q_ready(s))) break;
+                added |= issue_s(s);
+              } else {
+                if (lane == 0) mbar_arrive(&v_empty[st]);  // this tile does not read V at this k-tile
               }
-              umma_commit(&s_full[s]);
-              pkv[s] = kv_it;
-              const bool last = ++nS[s] == t[s].n;
-              pv |= (1u << s) | (nS[s] == 1 ? (4u << s) : 0u) | (last ? (16u << s) : 0u);
-              if (last) umma_commit(&q_empty[s]);  // last read of Q_s in this item
-            } else {
-              if (lane == 0) mbar_arrive(&v_empty[st]);  // this tile does not read V at this k-tile
+            }
+            if (!ok) break;
+#pragma unroll
+            for (int s = 0; s < 2; ++s)
+              if ((pv & (1u << s)) && !(ok = issue_pv(s))) break;
+            if (!ok) break;
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+              if (in[s]) {
+                pkv[s] = kv_it;
+                psq[s] = nsq[s] - 1;
+              }
+            }
+            pv |= added;
+          } else {
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+              if ((pv & (1u << s)) && !(ok = issue_pv(s))) break;
+              if (in[s]) {
+                if (!(ok = q_ready(s))) break;
+                pkv[s] = kv_it;
+                psq[s] = nsq[s];
+                pv |= issue_s(s);
+              } else {
+                if (lane == 0) mbar_arrive(&v_empty[st]);  // this tile does not read V at this k-tile
+              }
             }
           }
           if (!ok) break;
@@ -497,8 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sw = warp & 3;
     const int r = sw * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(sw * 32) << 16;
-    const uint32_t tmem_s = tmem + slot * BK;
-    const uint32_t tmem_o = tmem + 2 * BK + slot * D;
+    const uint32_t tmem_o = tmem + C::kOCol + slot * D;
     const MaskArgs& mk = p.mask;
     const bool k_ragged = (p.Nk % BK) != 0;
     int4* my_bounds = s_bounds + slot * 2 * BK;
@@ -594,7 +643,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (!(ok = warp_all(mbar_wait(&s_full[slot], s_cnt & 1, s_abort)))) break;
+        // S number s_cnt of this tile sits in buffer s_cnt % kSBufs.
+        const uint32_t sb = s_cnt % C::kSBufs;
+        const uint32_t tmem_s = tmem + (slot * C::kSBufs + sb) * BK;
+        if (!(ok = warp_all(mbar_wait(&s_full[2 * slot + sb], (s_cnt / C::kSBufs) & 1, s_abort)))) break;
         ++s_cnt;
         tc_fence_after();
 
@@ -647,7 +699,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_new;
         if (i > 0 && __any_sync(0xffffffffu, need)) {
           // Rare (the running max grew by more than the threshold): kept
-          // rolled to save instruction-cache space for the hot path.
+          // rolled to save instruction-cache space for the hot path. With two
+          // S buffers, S number k is issued before the P.V of S number k - 1,
+          // so that P.V (phase k - 1 of pv_done; at most one phase is pending)
+          // must complete before O is rescaled.
+          if (C::kSBufs == 2 && !(ok = warp_all(mbar_wait(&pv_done[slot], (s_cnt - 2) & 1, s_abort)))) break;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -661,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_full[slot]);
+        mbar_arrive(&p_full[2 * slot + sb]);
       }
       if (!ok) break;
 
