@@ -53,10 +53,15 @@ constexpr int kRows = 128;  // MMA M: query rows per tile
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 =
-// 64512); WG0 drops to 104 (the unrolled MMA issue must not spill) and the two
-// softmax warpgroups rise to 200: 128 x 104 + 256 x 200 = 64512.
-constexpr int kRegsLow = 104;
-constexpr int kRegsHigh = 200;
+// 64512), shared as 128 x low + 256 x high = 64512. With BK = 128 the softmax
+// holds a 128-score row and needs 200, leaving WG0 104; with BK = 64 it
+// needs far fewer and WG0 (the MMA warp with two S buffers) gets 120.
+template <int BK>
+constexpr int kRegsLow = BK == 64 ? 120 : 104;
+template <int BK>
+constexpr int kRegsHigh = BK == 64 ? 192 : 200;
+static_assert(128 * kRegsLow<64> + 256 * kRegsHigh<64> <= 384 * 168, "register split (BK = 64)");
+static_assert(128 * kRegsLow<128> + 256 * kRegsHigh<128> <= 384 * 168, "register split (BK = 128)");
 
 struct FwdParams {
   int32_t B, Hq, Hkv, G, Hm, Nq, Nk, nqt, nkt;
@@ -294,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *s_tmem;
 
   if (wg == 0) {
-   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(kRegsLow));
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(kRegsLow<BK>));
    if (warp == 0) {
     // =================== TMA producer ===================
     if (lane == 0) {
@@ -410,11 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // advancing by a byte offset adds offset >> 4 to the descriptor.
         // The MMAs are issued fully unrolled: a rolled issue loop costs about
         // twice the MMA's own 64 cycles per instruction.
-        const uint64_t vd = sdesc_sw128(v_addr + vst * C::kKVBytes, BK * 128, 1024);
+        const uint32_t vd = sdesc_sw128_lo(v_addr + vst * C::kKVBytes, BK * 128);
         umma_ts(d_o, a_p, vd, idesc_pv, (pv & (4u << s)) ? 0u : 1u);
 #pragma unroll
-        for (int kk = 1; kk < BK / 16; ++kk)
-          umma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * (16 * 128 / 16)), idesc_pv, 1u);
+        for (int kk = 1; kk < BK / 16; ++kk) umma_ts(d_o, a_p + kk * 8, vd + kk * (16 * 128 / 16), idesc_pv, 1u);
         // With one S buffer the next S of this slot is issued after this P.V,
         // so its s_full commit also covers this MMA; o_done is needed only
         // after the item's last P.V.
@@ -457,15 +461,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           // S_s = Q_s K^T for k-tile st; returns the pending-P.V flags it adds.
           auto issue_s = [&](int s) -> uint32_t {
             const uint32_t sb = nsq[s] % C::kSBufs;
-            const uint64_t qd = sdesc_sw128(q_addr + s * C::kQBytes, 16, 1024);
-            const uint64_t kd = sdesc_sw128(k_addr + st * C::kKVBytes, 16, 1024);
+            const uint32_t qd = sdesc_sw128_lo(q_addr + s * C::kQBytes, 16);
+            const uint32_t kd = sdesc_sw128_lo(k_addr + st * C::kKVBytes, 16);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               // K step of 16 bf16 = 32 bytes inside the 128-byte row; every 4
               // steps move to the next 64-column chunk of the tile.
               const uint32_t off = (kk & 3) * 32;
-              const uint64_t a = qd + static_cast<uint64_t>(((kk >> 2) * (kRows * 128) + off) >> 4);
-              const uint64_t bd = kd + static_cast<uint64_t>(((kk >> 2) * (BK * 128) + off) >> 4);
+              const uint32_t a = qd + (((kk >> 2) * (kRows * 128) + off) >> 4);
+              const uint32_t bd = kd + (((kk >> 2) * (BK * 128) + off) >> 4);
               umma_ss(tmem + (s * C::kSBufs + sb) * BK, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
             }
             umma_commit(&s_full[2 * s + sb]);
@@ -541,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
    }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(kRegsHigh));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(kRegsHigh<BK>));
     // =================== softmax / correction / epilogue ===================
     const int slot = wg - 1;
     const int sw = warp & 3;

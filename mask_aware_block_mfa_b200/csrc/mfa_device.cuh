@@ -215,28 +215,55 @@ __device__ __forceinline__ void tc_fence_after() {
 // cycles per 128x128x16 MMA in a steady stream, and a group of 8 MMAs from an
 // idle tensor pipe to its commit took 996 instead of 728 cycles.
 
-// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (bf16/f16 in, f32 accumulate).
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+// Shared-memory matrix descriptor, 128-byte swizzle (the layout TMA writes
+// with CU_TENSOR_MAP_SWIZZLE_128B). Bits: [0,14) start >> 4, [16,30) leading
+// byte offset >> 4, [32,46) stride byte offset >> 4, [46,48) version = 1,
+// [49,52) base offset = 0 (tiles are 1024-byte aligned), [61,64) layout = 2.
+//  K-major operand: rows of 128 bytes (64 bf16 along K), 8-row groups
+//    SBO = 1024 bytes apart; LBO unused (1). Advance K by 16 elements by adding
+//    32 bytes to the start address inside the 128-byte row.
+//  MN-major operand: 64 MN-contiguous elements per 128-byte row, K rows 128
+//    bytes apart, 8-row K groups SBO = 1024 bytes apart, 64-element MN chunks
+//    LBO bytes apart.
+// Every descriptor here has SBO = 1024, so its high word is the constant
+// kSdescHi and only the low word (start address and LBO) varies. The issue
+// helpers take that low word and rebuild the 64-bit operand inside the asm,
+// so the compiler keeps one register per descriptor instead of two across the
+// unrolled MMA groups (which made the MMA warp spill at its 104 registers).
+// Adding a byte offset >> 4 to the low word advances the start address (it
+// stays below 2^14: shared memory is under 256 KB).
+constexpr uint32_t kSdescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t sdesc_sw128_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16; A is M x K with two 16-bit
-// elements per 32-bit TMEM column (row i in lane i).
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (bf16/f16 in, f32
+// accumulate); the descriptors are given by their low words (sdesc_sw128_lo).
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                           uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 hi;\n\t.reg .b64 da, db;\n\t"
+      "mov.b32 hi, %5;\n\t"
+      "mov.b64 da, {%1, hi};\n\t"
+      "mov.b64 db, {%2, hi};\n\t"
       "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-      :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}"
+      :: "r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16; A is M x K with two 16-bit
+// elements per 32-bit TMEM column (row i in lane i); B by its low word.
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 hi;\n\t.reg .b64 db;\n\t"
+      "mov.b32 hi, %5;\n\t"
+      "mov.b64 db, {%2, hi};\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}"
+      :: "r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi)
       : "memory");
 }
 
@@ -283,26 +310,6 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
 // ------------------------------------------------------------------------
 // Descriptors
 // ------------------------------------------------------------------------
-// Shared-memory matrix descriptor, 128-byte swizzle (the layout TMA writes
-// with CU_TENSOR_MAP_SWIZZLE_128B). Bits: [0,14) start >> 4, [16,30) leading
-// byte offset >> 4, [32,46) stride byte offset >> 4, [46,48) version = 1,
-// [49,52) base offset = 0 (tiles are 1024-byte aligned), [61,64) layout = 2.
-//  K-major operand: rows of 128 bytes (64 bf16 along K), 8-row groups
-//    SBO = 1024 bytes apart; LBO unused (1). Advance K by 16 elements by adding
-//    32 bytes to the start address inside the 128-byte row.
-//  MN-major operand: 64 MN-contiguous elements per 128-byte row, K rows 128
-//    bytes apart, 8-row K groups SBO = 1024 bytes apart, 64-element MN chunks
-//    LBO bytes apart.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= static_cast<uint64_t>(1u) << 46;
-  d |= static_cast<uint64_t>(2u) << 61;
-  return d;
-}
-
 // Instruction descriptor, kind::f16 with bf16 A and B and an f32 accumulator:
 // [4,6) D format = 1 (F32), [7,10) A format = 1 (BF16), [10,13) B format = 1,
 // bit 15 A major (0 = K), bit 16 B major (1 = MN), [17,23) N >> 3, [24,29) M >> 4.
