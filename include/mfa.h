@@ -103,8 +103,9 @@ typedef struct {
  *   err        uint32 [4]: err[0] is the device error word (MFA_DEVERR_*
  *              bits), set by mfa_build_tile_map and mfa_fwd; err[1] and
  *              err[2] are mfa_fwd's work counters (the next work item and the
- *              number of finished CTAs), left at zero after every call. All
- *              four are cleared by mfa_build_tile_map. Because of the
+ *              number of finished CTAs), err[3] mfa_build_tile_map's count of
+ *              finished classification blocks; the counters are left at zero
+ *              after every call. All four are cleared by mfa_build_tile_map. Because of the
  *              counters, mfa_fwd calls that share one map must not overlap on
  *              the GPU (issue them on one stream, or order the streams).
  * Class rule for COLWISE / BAND with r0 = qt*block_q, r1 = min(r0+block_q, Nq):

@@ -8,13 +8,14 @@
 // column-wise row intervals (FlashMask's O(N) description), so the map costs
 // O(N) reads plus O(nqt * nkt) integer work, never an N x N mask.
 //
-// Three launches on the caller's stream:
+// Two launches on the caller's stream:
 //   k_tile_minmax    grid (nkt, B*Hm), block BK: per k-tile min/max of the
 //                    (normalised) bounds; validates them.
 //   k_tile_classify  grid (nqt, B*Hm), block 256: class of every (qt, kt),
-//                    ordered compaction of the non-SKIP kt, count.
-//   k_tile_order     one block: stable counting sort of the q-tiles by count,
-//                    largest first (the forward pass's work order).
+//                    ordered compaction of the non-SKIP kt, count; the block
+//                    that finishes last (a counter in err[3]) then sorts the
+//                    q-tiles by count, largest first (the forward pass's work
+//                    order), which saves a third launch per build.
 #include <climits>
 #include <cuda_runtime.h>
 
@@ -138,13 +139,53 @@ __device__ __forceinline__ int block_scan256(bool flag, int* s_warp, int* total)
   return before + in_warp;
 }
 
+// Stable counting sort of the E = B*Hm*nqt q-tiles by count, largest first,
+// by one block. Histogram and bucket offsets in shared memory (s_buf, nkt + 1
+// ints); warp 0 then places the entries 32 at a time in index order, so equal
+// counts keep ascending indices.
+__device__ void order_tiles(const int32_t* __restrict__ count, int E, int nkt, int32_t* __restrict__ order,
+                            int* s_buf) {
+  const int t = threadIdx.x;
+  for (int c = t; c <= nkt; c += blockDim.x) s_buf[c] = 0;
+  __syncthreads();
+  for (int e = t; e < E; e += blockDim.x) atomicAdd(&s_buf[count[e]], 1);
+  __syncthreads();
+  if (t == 0) {  // offsets for descending counts
+    int acc = 0;
+    for (int c = nkt; c >= 0; --c) {
+      const int h = s_buf[c];
+      s_buf[c] = acc;
+      acc += h;
+    }
+  }
+  __syncthreads();
+  if (t < 32) {
+    const int lane = t;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      const int c = e < E ? count[e] : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, c);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int leader = __ffs(peers) - 1;
+      int off = 0;
+      if (c >= 0 && lane == leader) off = s_buf[c];
+      off = __shfl_sync(0xffffffffu, off, leader);
+      if (c >= 0) order[off + rank] = e;
+      __syncwarp();
+      if (c >= 0 && lane == leader) s_buf[c] = off + __popc(peers);
+      __syncwarp();
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) k_tile_classify(MaskArgs m, int BQ, int BK, int nqt, int nkt,
                                                        const int32_t* __restrict__ kmm,
                                                        uint8_t* __restrict__ cls,
                                                        int32_t* __restrict__ list,
                                                        int32_t* __restrict__ count,
+                                                       int32_t* __restrict__ order,
                                                        uint32_t* __restrict__ err) {
-  extern __shared__ int s_sel[];  // BLOCKSEL: [BQ/64][sel_k]
+  extern __shared__ int s_sel[];  // BLOCKSEL: [BQ/64][sel_k]; then the order histogram
   __shared__ int s_warp[8];
   const int qt = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   const size_t e = static_cast<size_t>(bh) * nqt + qt;
@@ -219,45 +260,22 @@ __global__ void __launch_bounds__(256) k_tile_classify(MaskArgs m, int BQ, int B
   }
   if (t == 0) count[e] = running;
   for (int kt = running + t; kt < nkt; kt += 256) list[e * nkt + kt] = -1;
-}
 
-// Stable counting sort of the E = B*Hm*nqt q-tiles by count, largest first.
-// Histogram and bucket offsets in shared memory; one warp then places the
-// entries 32 at a time in index order so equal counts keep ascending indices.
-__global__ void __launch_bounds__(1024) k_tile_order(const int32_t* __restrict__ count, int E, int nkt,
-                                                     int32_t* __restrict__ order) {
-  extern __shared__ int s_buf[];  // hist/offset [nkt + 1]
-  const int t = threadIdx.x;
-  for (int c = t; c <= nkt; c += blockDim.x) s_buf[c] = 0;
-  __syncthreads();
-  for (int e = t; e < E; e += blockDim.x) atomicAdd(&s_buf[count[e]], 1);
-  __syncthreads();
-  if (t == 0) {  // offsets for descending counts
-    int acc = 0;
-    for (int c = nkt; c >= 0; --c) {
-      const int h = s_buf[c];
-      s_buf[c] = acc;
-      acc += h;
-    }
+  // The last block to finish (counter err[3], cleared with the error word at
+  // the start of the build) sorts the q-tiles; the fences order every block's
+  // count before its increment and the increments before the last block's
+  // reads.
+  __shared__ bool s_last;
+  if (t == 0) {
+    __threadfence();
+    const uint32_t n_blocks = gridDim.x * gridDim.y;
+    s_last = atomicAdd(&err[3], 1u) == n_blocks - 1;
   }
   __syncthreads();
-  if (t < 32) {
-    const int lane = t;
-    for (int base = 0; base < E; base += 32) {
-      const int e = base + lane;
-      const int c = e < E ? count[e] : -1;
-      const unsigned peers = __match_any_sync(0xffffffffu, c);
-      const int rank = __popc(peers & ((1u << lane) - 1u));
-      const int leader = __ffs(peers) - 1;
-      int off = 0;
-      if (c >= 0 && lane == leader) off = s_buf[c];
-      off = __shfl_sync(0xffffffffu, off, leader);
-      if (c >= 0) order[off + rank] = e;
-      __syncwarp();
-      if (c >= 0 && lane == leader) s_buf[c] = off + __popc(peers);
-      __syncwarp();
-    }
-  }
+  if (!s_last) return;
+  __threadfence();
+  order_tiles(count, static_cast<int>(gridDim.y) * nqt, nkt, order, s_sel);
+  if (t == 0) err[3] = 0;
 }
 
 }  // namespace
@@ -285,15 +303,15 @@ extern "C" mfa_status mfa_build_tile_map(const mfa_mask_desc* mask, mfa_tile_map
   if (map->nqt > 0) {
     const size_t sel_smem =
         mask->kind == MFA_MASK_BLOCKSEL ? static_cast<size_t>(map->block_q / kSelBlock) * mask->sel_k * sizeof(int) : 0;
-    k_tile_classify<<<dim3(map->nqt, BH), 256, sel_smem, s>>>(m, map->block_q, map->block_k, map->nqt,
-                                                               map->nkt, map->kminmax, map->tile_class,
-                                                               map->tile_list, map->tile_count, map->err);
     const size_t ord_smem = static_cast<size_t>(map->nkt + 1) * sizeof(int);
-    if (ord_smem > 48 * 1024 &&
-        cudaFuncSetAttribute(k_tile_order, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(ord_smem)) != cudaSuccess)
+    const size_t smem = sel_smem > ord_smem ? sel_smem : ord_smem;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(k_tile_classify, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
       return MFA_ERR_CUDA;
-    k_tile_order<<<1, 1024, ord_smem, s>>>(map->tile_count, BH * map->nqt, map->nkt, map->order);
+    k_tile_classify<<<dim3(map->nqt, BH), 256, smem, s>>>(m, map->block_q, map->block_k, map->nqt, map->nkt,
+                                                           map->kminmax, map->tile_class, map->tile_list,
+                                                           map->tile_count, map->order, map->err);
   }
   return cudaGetLastError() == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
 }
