@@ -357,7 +357,7 @@ def main():
                      "peak_kind": f"{src} burst bf16 dense"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms": statistics.mean(e2e_ms)},
-        "gpu_launches": 4 * args.steps,  # per step: 3 tile-map kernels + 1 forward kernel
+        "gpu_launches": 3 * args.steps,  # per step: 2 tile-map kernels + 1 forward kernel
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline and world == 1:
