@@ -254,6 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   WorkItem* ring = reinterpret_cast<WorkItem*>(smem + C::kRingOff);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
+  uint32_t* s_epi = reinterpret_cast<uint32_t*>(smem + C::kMisc + 8);  // tile 0's finished epilogue warps
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wg = warp >> 2;
@@ -284,6 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sched_empty[i], 1 + 8);  // the MMA thread and one lane of each softmax warp
     }
     *s_abort = 0;
+    *s_epi = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -556,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool k_ragged = (p.Nk % BK) != 0;
     int4* my_bounds = s_bounds + slot * 2 * BK;
     uint64_t* my_bnd = bnd_full + 2 * slot;
-    uint32_t s_cnt = 0, o_cnt = 0, n_bnd = 0;
+    uint32_t s_cnt = 0, o_cnt = 0, n_bnd = 0, epi_items = 0;
     bool ok = true;
 
     for (int it = 0; ok; ++it) {
@@ -738,6 +740,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool store = qi < p.Nq;
       __nv_bfloat16* orow = p.out + static_cast<int64_t>(T.b) * p.os0 + static_cast<int64_t>(head) * p.os1 +
                             static_cast<int64_t>(qi) * p.os2;
+      // In kind-0 items both tiles finish together and their row stores would
+      // share the load/store unit; tile 1 stores after tile 0 has issued its
+      // stores, so tile 0 goes on to its next item earlier and the tiles end up
+      // staggered. The count of tile 0's finished warps only grows, so a wait
+      // cannot confuse one item with another; the spin is bounded.
+      if (slot == 1 && p.item_kind == 0) {
+        const uint32_t want = 4u * ++epi_items;
+        uint64_t t0 = 0;
+        for (uint32_t k = 0; *reinterpret_cast<volatile uint32_t*>(s_epi) < want; ++k) {
+          if ((k & 255) == 255) {
+            if (t0 == 0) t0 = global_timer_ns();
+            if (*s_abort || global_timer_ns() - t0 > kWaitTimeoutNs) {
+              *s_abort = 1;
+              ok = false;
+              break;
+            }
+          }
+        }
+        if (!(ok = warp_all(ok))) break;
+      }
       // Each thread writes its own row. With 32-byte aligned rows a store
       // covers whole 32-byte sectors; 16-byte stores would write every sector
       // in two halves from two instructions. The chunk loop stays rolled: it
@@ -767,6 +789,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (store) {
         const float lse = has ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
         p.lse[(static_cast<size_t>(T.b) * p.Hq + head) * p.Nq + qi] = lse;
+      }
+      if (slot == 0 && p.item_kind == 0) {
+        __syncwarp();
+        if (lane == 0) atomicAdd(s_epi, 1u);
       }
     }
     if (!ok && lane == 0) atomicOr(p.err, MFA_DEVERR_TIMEOUT);
