@@ -79,7 +79,10 @@ def attention(q, k, v, mask, rows: Optional[Sequence[int]] = None,
         for hi, h in enumerate(heads):
             hm = 0 if mask.Hm == 1 else h
             if hm not in vis_cache:
-                vis_cache[hm] = masks.visible_rows(mask, b, hm, rows)
+                if hasattr(mask, "visible_rows"):  # e.g. sparse_modes.SparseMode
+                    vis_cache[hm] = mask.visible_rows(b, hm, rows)
+                else:
+                    vis_cache[hm] = masks.visible_rows(mask, b, hm, rows)
             o, s = attention_rows(q[b, h, rows], k[b, h // G], v[b, h // G], vis_cache[hm])
             out[bi, hi], lse[bi, hi] = o, s
     return out, lse
