@@ -158,8 +158,56 @@ mfa_status mfa_tile_map_init(mfa_tile_map* map, void* device_buf, size_t bytes,
                              int32_t B, int32_t Hm, int32_t Nq, int32_t Nk,
                              int32_t block_q, int32_t block_k);
 
+/* Ascend sparse modes (Ascend CANN "sparseMode introduction" page, one
+ * paragraph per mode) as a compact mask description. Rows are queries [0, Nq), columns
+ * keys [0, Nk); d = Nk - Nq.
+ *   0 defaultMask   band -pre <= j - i <= next, origin at the upper left
+ *   2 leftUpCausal  j <= i
+ *   3 rightDownCausal  j - i <= d
+ *   4 band from the lower-right vertex: -pre <= (j - i) - d <= next
+ *   5, 6 prefix     j < prefix[b] or j - i <= d (6 differs from 5 only in the
+ *                   page's attenMask input format)
+ *   7, 8 varlen, long sequence split externally: B = 1 packs n_seq sequences
+ *                   with cumulative query ends seq_q (actual_seq_qlen) and key
+ *                   ends seq_kv (actual_seq_kvlen); pairs of different
+ *                   sequences are masked. Inside a sequence of lengths (lq, lk):
+ *                   mode 7 is rightDownCausal except the last non-empty
+ *                   sequence, mode 8 leftUpCausal except the first non-empty
+ *                   one, which take the band from the sequence's lower-right
+ *                   vertex with (pre, next).
+ * Mode 1 (a full attenMask) has no compact form: MFA_ERR_UNSUPPORTED. */
+typedef struct mfa_sparse_mode {
+  int32_t mode;
+  int32_t reserved;                /* 0 */
+  int64_t pre_tokens, next_tokens; /* modes 0, 4, 7, 8 */
+  const int64_t* prefix;           /* modes 5, 6: DEVICE [B] prefix lengths */
+  const int64_t* seq_q;            /* modes 7, 8: DEVICE [n_seq] cumulative query ends */
+  const int64_t* seq_kv;           /* modes 7, 8: DEVICE [n_seq] cumulative key ends */
+  int32_t n_seq;                   /* modes 7, 8: number of packed sequences (>= 1) */
+  int32_t reserved2;               /* 0 */
+} mfa_sparse_mode;
+
+/* Fill *out (kind, B, Hm = 1, Nq, Nk and the kind's fields; out->map is left
+ * NULL) for the sparse mode `sm`, the library's mask description for it.
+ *   Modes 0, 2, 3, 4 become MFA_MASK_BAND with the tokens shifted to the
+ *   upper-left origin (pre - d, next + d for mode 4); nothing is launched and
+ *   the four arrays may be NULL.
+ *   Modes 5-8 become MFA_MASK_COLWISE: one kernel writes the caller-owned
+ *   DEVICE int32 arrays lts, lte, uts, ute [B, 1, Nk] on `stream` (every key
+ *   column needs at most the two masked row intervals of that format). The
+ *   description points at those arrays, which must outlive its use.
+ *   Prefix lengths and cumulative ends are clamped to [0, Nk] / [0, Nq], and
+ *   tokens to +-(Nq + Nk + 1); the cumulative ends must not decrease (the
+ *   key column of a sequence is found by binary search). Keys past the last
+ *   sequence are masked for every query.
+ * Errors: MFA_ERR_INVALID_ARG (NULL sm/out, shapes < 0, B > 65535, B != 1 or n_seq < 1
+ * for modes 7, 8, missing arrays), MFA_ERR_UNSUPPORTED (mode 1 or unknown),
+ * MFA_ERR_CUDA (launch failure). */
+mfa_status mfa_mask_from_sparse_mode(const mfa_sparse_mode* sm, int32_t B, int32_t Nq, int32_t Nk, int32_t* lts,
+                                     int32_t* lte, int32_t* uts, int32_t* ute, mfa_mask_desc* out, void* stream);
+
 /* Build `map` from `mask` on `stream`: clears err, computes kminmax,
- * tile_class, tile_list, tile_count and order (three kernel launches). The
+ * tile_class, tile_list, tile_count and order (two kernel launches). The
  * mask's shape must equal the map's. mask->map is ignored. Device-detected
  * range errors set MFA_DEVERR_BOUNDS / MFA_DEVERR_SEL. */
 mfa_status mfa_build_tile_map(const mfa_mask_desc* mask, mfa_tile_map* map, void* stream);

@@ -23,7 +23,8 @@ MFA_BF16, MFA_F32 = 0, 1
 DEVERR_BOUNDS, DEVERR_SEL, DEVERR_TIMEOUT, DEVERR_MAP = 1, 2, 4, 8
 
 EXPORTS = ("mfa_abi_version", "mfa_status_string", "mfa_tile_map_bytes", "mfa_tile_map_init",
-           "mfa_build_tile_map", "mfa_fwd", "mfa_fwd_noalloc", "mfa_get_device_status")
+           "mfa_build_tile_map", "mfa_fwd", "mfa_fwd_noalloc", "mfa_get_device_status",
+           "mfa_mask_from_sparse_mode")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -48,6 +49,13 @@ class MfaMaskDesc(ctypes.Structure):
                 ("lts", ctypes.c_void_p), ("lte", ctypes.c_void_p), ("uts", ctypes.c_void_p), ("ute", ctypes.c_void_p),
                 ("pre_tokens", ctypes.c_int64), ("next_tokens", ctypes.c_int64),
                 ("sel", ctypes.c_void_p), ("map", ctypes.POINTER(MfaTileMap))]
+
+
+class MfaSparseMode(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("pre_tokens", ctypes.c_int64), ("next_tokens", ctypes.c_int64),
+                ("prefix", ctypes.c_void_p), ("seq_q", ctypes.c_void_p), ("seq_kv", ctypes.c_void_p),
+                ("n_seq", ctypes.c_int32), ("reserved2", ctypes.c_int32)]
 
 
 class MfaError(RuntimeError):
@@ -87,6 +95,9 @@ def load(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.mfa_get_device_status.restype = ctypes.c_int
     lib.mfa_get_device_status.argtypes = [ctypes.POINTER(MfaTileMap), ctypes.c_void_p,
                                           ctypes.POINTER(ctypes.c_uint32)]
+    lib.mfa_mask_from_sparse_mode.restype = ctypes.c_int
+    lib.mfa_mask_from_sparse_mode.argtypes = [ctypes.POINTER(MfaSparseMode)] + [ctypes.c_int32] * 3 + \
+        [ctypes.c_void_p] * 4 + [ctypes.POINTER(MfaMaskDesc), ctypes.c_void_p]
     if lib.mfa_abi_version() != 1:
         raise RuntimeError("libmfa.so ABI version mismatch")
     _lib = lib
@@ -143,6 +154,37 @@ class DeviceMask:
         d.pre_tokens, d.next_tokens = int(mask.pre_tokens), int(mask.next_tokens)
         d.map = None
         self.desc = d
+
+
+class SparseModeMask:
+    """An Ascend sparse mode turned into a device mask description by
+    mfa_mask_from_sparse_mode (band modes on the host, prefix and varlen modes
+    by a kernel into column-wise bounds owned here). Usable wherever a
+    DeviceMask is (build_tile_map, fwd, Attention)."""
+
+    def __init__(self, mode: int, B: int, Nq: int, Nk: int, pre_tokens: int = 0, next_tokens: int = 0,
+                 prefix=None, seq_q=None, seq_kv=None, device="cuda", stream=None):
+        self.B, self.Hm, self.Nq, self.Nk = B, 1, Nq, Nk
+        self._keep = []
+        sm = MfaSparseMode()
+        sm.mode, sm.pre_tokens, sm.next_tokens = mode, int(pre_tokens), int(next_tokens)
+
+        def dev64(a):
+            if a is None:
+                return None
+            t = torch.as_tensor(np.asarray(a, dtype=np.int64)).to(device)
+            self._keep.append(t)
+            return t.data_ptr()
+
+        sm.prefix, sm.seq_q, sm.seq_kv = dev64(prefix), dev64(seq_q), dev64(seq_kv)
+        sm.n_seq = 0 if seq_q is None else len(seq_q)
+        self.bounds = torch.empty(4, max(B, 1), 1, max(Nk, 1), dtype=torch.int32, device=device)
+        ptrs = [self.bounds[i].data_ptr() for i in range(4)]  # lts, lte, uts, ute
+        self.desc = MfaMaskDesc()
+        _check("mfa_mask_from_sparse_mode",
+               load().mfa_mask_from_sparse_mode(ctypes.byref(sm), B, Nq, Nk, *ptrs, ctypes.byref(self.desc),
+                                                _stream_ptr(stream)))
+        self.kind = self.desc.kind
 
 
 class TileMap:
@@ -222,8 +264,9 @@ def device_status(tmap: TileMap, stream=None) -> int:
 class Attention:
     """Convenience wrapper: upload a mask, build its map once, run forward passes."""
 
-    def __init__(self, mask: W.MaskDesc, block_q: int = 64, block_k: int = 128, device="cuda"):
-        self.dmask = DeviceMask(mask, device)
+    def __init__(self, mask, block_q: int = 64, block_k: int = 128, device="cuda"):
+        # a workloads.MaskDesc (uploaded here) or a mask already on the device
+        self.dmask = DeviceMask(mask, device) if isinstance(mask, W.MaskDesc) else mask
         self.tmap = TileMap(mask.B, mask.Hm, mask.Nq, mask.Nk, block_q, block_k, device)
         self.device = device
 

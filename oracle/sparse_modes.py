@@ -1,7 +1,7 @@
 """Dense visibility of the Ascend sparse modes (oracle; test infrastructure).
 
-Written from the Ascend FlashAttentionScore page, "sparseMode" paragraphs and
-their worked examples. Rows are queries i in [0, Sq), columns keys j in
+Written from the Ascend CANN "sparseMode introduction" page (one paragraph
+per mode) and its worked examples. Rows are queries i in [0, Sq), columns keys j in
 [0, Skv); True means the pair is computed (attenMask False). Each mode is
 coded from its own sentence, independently of the library's conversion of
 the mode into a compact mask description:

@@ -47,8 +47,9 @@ def test_struct_layouts_match_header(tmp_path):
 #include "mfa.h"
 #define F(T, f) printf(#T "." #f " %zu\n", offsetof(T, f))
 int main(void) {
-  printf("mfa_tensor %zu\nmfa_tile_map %zu\nmfa_mask_desc %zu\n",
-         sizeof(mfa_tensor), sizeof(mfa_tile_map), sizeof(mfa_mask_desc));
+  printf("mfa_tensor %zu\nmfa_tile_map %zu\nmfa_mask_desc %zu\nmfa_sparse_mode %zu\n",
+         sizeof(mfa_tensor), sizeof(mfa_tile_map), sizeof(mfa_mask_desc), sizeof(mfa_sparse_mode));
+  F(mfa_sparse_mode, pre_tokens); F(mfa_sparse_mode, prefix); F(mfa_sparse_mode, seq_kv); F(mfa_sparse_mode, n_seq);
   F(mfa_tensor, data); F(mfa_tensor, B); F(mfa_tensor, stride);
   F(mfa_tile_map, kind); F(mfa_tile_map, kminmax); F(mfa_tile_map, err);
   F(mfa_mask_desc, lts); F(mfa_mask_desc, pre_tokens); F(mfa_mask_desc, sel); F(mfa_mask_desc, map);
@@ -60,10 +61,12 @@ int main(void) {
     assert int(got["mfa_tensor"]) == ctypes.sizeof(B.MfaTensor)
     assert int(got["mfa_tile_map"]) == ctypes.sizeof(B.MfaTileMap)
     assert int(got["mfa_mask_desc"]) == ctypes.sizeof(B.MfaMaskDesc)
+    assert int(got["mfa_sparse_mode"]) == ctypes.sizeof(B.MfaSparseMode)
     for key, val in got.items():
         if "." in key:
             struct, field = key.split(".")
-            cls = {"mfa_tensor": B.MfaTensor, "mfa_tile_map": B.MfaTileMap, "mfa_mask_desc": B.MfaMaskDesc}[struct]
+            cls = {"mfa_tensor": B.MfaTensor, "mfa_tile_map": B.MfaTileMap, "mfa_mask_desc": B.MfaMaskDesc,
+                   "mfa_sparse_mode": B.MfaSparseMode}[struct]
             assert getattr(cls, field).offset == int(val), key
 
 

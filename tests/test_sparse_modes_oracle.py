@@ -1,6 +1,6 @@
 """The oracle's Ascend sparse modes against closed forms and the page's examples.
 
-Pins (Ascend FlashAttentionScore page, "sparseMode"):
+Pins (Ascend CANN "sparseMode introduction" page):
 * square shapes: modes 2 and 3 are the plain causal triangle and mode 4 is
   mode 0 (the page: the lower-right and upper-left origins coincide);
 * per-row visible counts in closed form for modes 0, 2, 3, 4 and 5 on
