@@ -41,6 +41,7 @@ BLOCKS = {  # launch configuration per workload: (block_q, block_k)
     "band16k_neg": (128, 128),
     "doc32k": (64, 128),
     "blocksel32k": (64, 64),
+    "varlen_prefill16k": (64, 128),
 }
 METRIC = "effective TFLOP/s (visible pairs only) and % of B200 bf16 tensor peak"
 
@@ -78,8 +79,36 @@ def peaks():
         return 1590.0, 1400.0, "fallback"
 
 
+def sparse_mode_pairs(m) -> int:
+    """Visible pairs of the varlen sparse modes from the page's per-sequence
+    rules: rightDownCausal (7) or leftUpCausal (8) inside each packed sequence,
+    the band from the sequence's lower-right vertex for the last (7) or first
+    (8) non-empty one."""
+    if m.mode not in (7, 8):
+        raise ValueError("bench workloads use sparse modes 7 and 8 only")
+    ends_q = [0] + [int(x) for x in m.seq_q]
+    ends_k = [0] + [int(x) for x in m.seq_kv]
+    seqs = [(ends_q[s + 1] - ends_q[s], ends_k[s + 1] - ends_k[s]) for s in range(len(m.seq_q))]
+    nonempty = [s for s, (lq, lk) in enumerate(seqs) if lq > 0 and lk > 0]
+    band = (nonempty[-1] if m.mode == 7 else nonempty[0]) if nonempty else -1
+    total = 0
+    for s, (lq, lk) in enumerate(seqs):
+        li = np.arange(lq, dtype=np.int64)
+        if s == band:
+            lo = np.maximum(li + (lk - lq) - int(m.pre_tokens), 0)
+            hi = np.minimum(li + (lk - lq) + int(m.next_tokens), lk - 1)
+        elif m.mode == 7:
+            lo, hi = np.zeros_like(li), np.minimum(li + (lk - lq), lk - 1)
+        else:
+            lo, hi = np.zeros_like(li), np.minimum(li, lk - 1)
+        total += int(np.maximum(hi - lo + 1, 0).sum())
+    return total
+
+
 def visible_pairs(mask) -> int:
     """Visible pairs from the description's own closed forms (host integer arithmetic)."""
+    if isinstance(mask, W.SparseModeInput):
+        return sparse_mode_pairs(mask)
     total = 0
     for b in range(mask.B):
         if mask.kind == W.MASK_BAND:
@@ -162,16 +191,25 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def oracle_mask(mask):
+    """The mask as the oracle takes it (sparse-mode inputs become the oracle's own mode object)."""
+    if isinstance(mask, W.SparseModeInput):
+        from oracle import sparse_modes as SM
+        return SM.SparseMode(**mask.fields())
+    return mask
+
+
 def run_reference(args, prob, pairs, d, Hq):
     """The reference arm: the float64 CPU oracle, each step a bounded sample of the workload."""
     from threadpoolctl import threadpool_info
     from oracle import attention as OA
     heads = list(range(min(args.reference_heads, Hq)))
     flops = 4.0 * d * pairs * len(heads) / (1 if prob.mask.Hm == 1 else Hq)
+    omask = oracle_mask(prob.mask)
     times = []
     for s in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        OA.attention(prob.q, prob.k, prob.v, prob.mask, heads=heads)
+        OA.attention(prob.q, prob.k, prob.v, omask, heads=heads)
         if s >= args.warmup:
             times.append(time.perf_counter() - t0)
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -192,8 +230,9 @@ def cpu_baseline(prob, pairs, d, Hq, heads_n):
     from threadpoolctl import threadpool_info
     from oracle import attention as OA
     heads = list(range(min(heads_n, Hq)))
+    omask = oracle_mask(prob.mask)
     t0 = time.perf_counter()
-    OA.attention(prob.q, prob.k, prob.v, prob.mask, heads=heads)
+    OA.attention(prob.q, prob.k, prob.v, omask, heads=heads)
     sec = time.perf_counter() - t0
     flops = 4.0 * d * pairs * len(heads) / (1 if prob.mask.Hm == 1 else Hq)
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -239,13 +278,23 @@ def main():
 
     bq, bk = BLOCKS[args.workload]
     q, k, v = (t.to(dev) for t in (prob.q, prob.k, prob.v))
-    att = B.Attention(prob.mask, bq, bk, device=dev)
+    sparse = isinstance(prob.mask, W.SparseModeInput)
+
+    def device_mask(stream=None):
+        """Mask arrays host -> device (and, for a sparse mode, its conversion kernel)."""
+        if sparse:
+            return B.SparseModeMask(**prob.mask.fields(), device=dev, stream=stream)
+        return B.DeviceMask(prob.mask, dev)
+
+    att = B.Attention(device_mask(), bq, bk, device=dev)
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
+        if sparse:
+            att.dmask.convert()
         att.build()
         att(q, k, v, out, lse)
 
@@ -311,8 +360,8 @@ def main():
     hq, hk, hv = (t.pin_memory() for t in (prob.q, prob.k, prob.v))
     ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    mask_bytes = sum(getattr(prob.mask, f).nbytes for f in ("lts", "lte", "uts", "ute", "sel")
-                     if getattr(prob.mask, f) is not None)
+    mask_fields = ("prefix", "seq_q", "seq_kv") if sparse else ("lts", "lte", "uts", "ute", "sel")
+    mask_bytes = sum(getattr(prob.mask, f).nbytes for f in mask_fields if getattr(prob.mask, f) is not None)
     h2d = hq.nbytes + hk.nbytes + hv.nbytes + mask_bytes
     d2h = ho.nbytes + hl.nbytes
     e2e_ms = []
@@ -321,7 +370,7 @@ def main():
         z = torch.cuda.Event(enable_timing=True)
         a.record(stream)
         att_e = att
-        att_e.dmask = B.DeviceMask(prob.mask, dev)  # mask arrays host -> device
+        att_e.dmask = device_mask(stream)
         q.copy_(hq, non_blocking=True)
         k.copy_(hk, non_blocking=True)
         v.copy_(hv, non_blocking=True)
@@ -345,9 +394,10 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, "desc": W.WORKLOADS[args.workload], "B": Bsz, "Hq": Hq, "Hkv": Hkv,
-                   "N": N, "d": d, "block_q": bq, "block_k": bk, "seed": prob.seed, "visible_pairs": pairs,
+                   "N": N, "Nk": prob.Nk, "d": d, "block_q": bq, "block_k": bk, "seed": prob.seed, "visible_pairs": pairs,
                    "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}",
-                   "launch": "each step replayed as a CUDA graph (map build + forward)"},
+                   "launch": "each step replayed as a CUDA graph (" + ("sparse-mode conversion + " if sparse else "")
+                             + "map build + forward)"},
         "frac_of_peak": {"burst": value / burst, "sustained": value / sustained, "spec_2250": value / 2250.0,
                          "peaks": src},
         "fwd_only": {"ms": fwd_avg_ms, "tflops": achieved},
@@ -357,7 +407,8 @@ def main():
                      "peak_kind": f"{src} burst bf16 dense"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms": statistics.mean(e2e_ms)},
-        "gpu_launches": 3 * args.steps,  # per step: 2 tile-map kernels + 1 forward kernel
+        # per step: 2 tile-map kernels + 1 forward kernel (+1 sparse-mode conversion kernel)
+        "gpu_launches": (4 if sparse and prob.mask.mode >= 5 else 3) * args.steps,
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline and world == 1:

@@ -139,6 +139,7 @@ class DeviceMask:
 
     def __init__(self, mask: W.MaskDesc, device="cuda"):
         self.mask = mask
+        self.kind, self.B, self.Hm, self.Nq, self.Nk = mask.kind, mask.B, mask.Hm, mask.Nq, mask.Nk
         self._keep = []
         d = MfaMaskDesc()
         d.kind, d.B, d.Hm, d.Nq, d.Nk = mask.kind, mask.B, mask.Hm, mask.Nq, mask.Nk
@@ -178,13 +179,19 @@ class SparseModeMask:
 
         sm.prefix, sm.seq_q, sm.seq_kv = dev64(prefix), dev64(seq_q), dev64(seq_kv)
         sm.n_seq = 0 if seq_q is None else len(seq_q)
+        self.sm = sm
         self.bounds = torch.empty(4, max(B, 1), 1, max(Nk, 1), dtype=torch.int32, device=device)
-        ptrs = [self.bounds[i].data_ptr() for i in range(4)]  # lts, lte, uts, ute
         self.desc = MfaMaskDesc()
-        _check("mfa_mask_from_sparse_mode",
-               load().mfa_mask_from_sparse_mode(ctypes.byref(sm), B, Nq, Nk, *ptrs, ctypes.byref(self.desc),
-                                                _stream_ptr(stream)))
+        self.convert(stream)
         self.kind = self.desc.kind
+
+    def convert(self, stream=None) -> None:
+        """(Re)write the description, and for modes 5-8 the bounds, from the
+        mode's inputs already on the device (no allocation, graph-capturable)."""
+        ptrs = [self.bounds[i].data_ptr() for i in range(4)]  # lts, lte, uts, ute
+        _check("mfa_mask_from_sparse_mode",
+               load().mfa_mask_from_sparse_mode(ctypes.byref(self.sm), self.B, self.Nq, self.Nk, *ptrs,
+                                                ctypes.byref(self.desc), _stream_ptr(stream)))
 
 
 class TileMap:

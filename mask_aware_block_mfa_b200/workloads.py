@@ -60,20 +60,49 @@ class MaskDesc:
 
 
 @dataclasses.dataclass
+class SparseModeInput:
+    """The inputs of an Ascend sparse mode (mode number, tokens, prefix lengths
+    or cumulative sequence ends), kept as drawn. The CUDA path turns it into a
+    compact description with mfa_mask_from_sparse_mode; the oracle expands the
+    same numbers itself."""
+
+    mode: int
+    B: int
+    Nq: int
+    Nk: int
+    pre_tokens: int = 0
+    next_tokens: int = 0
+    prefix: Optional[np.ndarray] = None  # int64 [B]
+    seq_q: Optional[np.ndarray] = None   # int64 [n_seq], cumulative query ends
+    seq_kv: Optional[np.ndarray] = None  # int64 [n_seq], cumulative key ends
+    Hm: int = 1
+    name: str = ""
+
+    def fields(self) -> dict:
+        return dict(mode=self.mode, B=self.B, Nq=self.Nq, Nk=self.Nk, pre_tokens=self.pre_tokens,
+                    next_tokens=self.next_tokens, prefix=self.prefix, seq_q=self.seq_q, seq_kv=self.seq_kv)
+
+
+@dataclasses.dataclass
 class Problem:
-    """One attention problem: q [B,Hq,N,d], k/v [B,Hkv,N,d] and its mask."""
+    """One attention problem: q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] and its mask
+    (a compact description, or the inputs of an Ascend sparse mode)."""
 
     name: str
     q: torch.Tensor
     k: torch.Tensor
     v: torch.Tensor
-    mask: MaskDesc
+    mask: object  # MaskDesc or SparseModeInput
     seed: int
 
     @property
     def shape(self):
         B, Hq, N, d = self.q.shape
         return B, Hq, int(self.k.shape[1]), N, d
+
+    @property
+    def Nk(self) -> int:
+        return int(self.k.shape[2])
 
 
 # ----------------------------------------------------------------------------
@@ -184,12 +213,14 @@ def _as_desc_arrays(m: MaskDesc) -> MaskDesc:
 # Tensors
 # ----------------------------------------------------------------------------
 
-def randn_qkv(seed: int, B: int, Hq: int, Hkv: int, N: int, d: int, dtype=torch.bfloat16):
+def randn_qkv(seed: int, B: int, Hq: int, Hkv: int, N: int, d: int, dtype=torch.bfloat16,
+              Nk: Optional[int] = None):
+    Nk = N if Nk is None else Nk
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     q = torch.randn((B, Hq, N, d), generator=g, dtype=torch.float32)
-    k = torch.randn((B, Hkv, N, d), generator=g, dtype=torch.float32)
-    v = torch.randn((B, Hkv, N, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
     return q.to(dtype), k.to(dtype), v.to(dtype)
 
 
@@ -205,6 +236,9 @@ WORKLOADS = {
     "band16k_neg": "B=2 Hq=Hkv=16 d=128 N=16384 bf16; band preTokens=4096 nextTokens=-64",
     "doc32k": "B=1 Hq=32 Hkv=8 d=128 N=32768 bf16; causal document mask, 8..32 documents",
     "blocksel32k": "B=1 Hq=32 Hkv=8 d=128 N=32768 bf16; top-16 of 64-key blocks per 64-query block",
+    "varlen_prefill16k": "B=1 Hq=32 Hkv=8 d=128 Nk=16384 Nq~8K bf16; sparseMode 7, packed sequences "
+                         "of 64*U{8..64} keys whose second halves are the queries (rightDownCausal; the last "
+                         "sequence as the band preTokens=its length, nextTokens=0)",
 }
 
 SEEDS = {
@@ -215,6 +249,7 @@ SEEDS = {
     "band16k_neg": 4001,
     "doc32k": 5000,
     "blocksel32k": 5001,
+    "varlen_prefill16k": 6000,
 }
 
 
@@ -256,7 +291,23 @@ def make_mask(name: str, seed: Optional[int] = None, N: Optional[int] = None) ->
     if name == "blocksel32k":
         N = 32768 if N is None else N
         return blocksel_topk(rng, 1, N, 16, name)
+    if name == "varlen_prefill16k":
+        return varlen_prefill(rng, 16384 if N is None else N, name)
     raise KeyError(name)
+
+
+def varlen_prefill(rng: np.random.Generator, Nk: int, name: str = "") -> SparseModeInput:
+    """Packed chunked prefill under sparseMode 7: sequences of 64*U{8..64} keys
+    (the last cut to fit Nk); each sequence's queries are its last
+    max(64, half rounded down to 64) tokens. The last sequence is the band with
+    preTokens = its key length and nextTokens = 0, the page's setting for a
+    split rightDownCausal sequence."""
+    lk = doc_lengths_uniform(rng, Nk, 8, 64)
+    lq = [max(64, (n // 2) // 64 * 64) if n >= 64 else n for n in lk]
+    seq_kv = np.cumsum(lk).astype(np.int64)
+    seq_q = np.cumsum(lq).astype(np.int64)
+    return SparseModeInput(7, 1, int(seq_q[-1]), int(seq_kv[-1]), pre_tokens=int(lk[-1]), next_tokens=0,
+                           seq_q=seq_q, seq_kv=seq_kv, name=name)
 
 
 SHAPES = {
@@ -268,6 +319,7 @@ SHAPES = {
     "band16k_neg": (2, 16, 16, 16384, 128, torch.bfloat16),
     "doc32k": (1, 32, 8, 32768, 128, torch.bfloat16),
     "blocksel32k": (1, 32, 8, 32768, 128, torch.bfloat16),
+    "varlen_prefill16k": (1, 32, 8, 16384, 128, torch.bfloat16),  # N = Nk; Nq from the draw
 }
 
 
@@ -279,7 +331,11 @@ def make_problem(name: str, seed: Optional[int] = None, N: Optional[int] = None,
     N = n if N is None else N
     Hq = hq if Hq is None else Hq
     Hkv = hkv if Hkv is None else Hkv
-    mask = _as_desc_arrays(make_mask(name, seed, N))
+    mask = make_mask(name, seed, N)
+    if isinstance(mask, SparseModeInput):
+        q, k, v = randn_qkv(seed + 17, B, Hq, Hkv, mask.Nq, d, dtype, Nk=mask.Nk)
+        return Problem(name, q, k, v, mask, seed)
+    mask = _as_desc_arrays(mask)
     q, k, v = randn_qkv(seed + 17, B, Hq, Hkv, N, d, dtype)
     return Problem(name, q, k, v, mask, seed)
 

@@ -31,3 +31,23 @@ def test_ncu_traffic_follows_the_kernel_digest():
     for name, (nbytes, dig) in bench.NCU_TRAFFIC.items():
         assert nbytes > 0 and len(dig) == 16
         assert bench.ncu_traffic(name) == (nbytes if dig == digest else None)
+
+
+@pytest.mark.parametrize("N", [2048, 5000, None])
+def test_varlen_prefill_pairs_match_the_oracle_modes(N):
+    from oracle import sparse_modes as SM
+    m = W.make_mask("varlen_prefill16k", N=N)
+    assert m.Nq < m.Nk and m.seq_kv[-1] == m.Nk and m.seq_q[-1] == m.Nq
+    ref = SM.SparseMode(**m.fields())
+    assert bench.visible_pairs(m) == int(SM.visible_dense(ref).sum())
+    # the band of the last sequence (pre = its key length, next = 0) equals its rightDownCausal triangle
+    diag = W.SparseModeInput(**{**m.fields(), "pre_tokens": 0, "next_tokens": 0})
+    lk = int(m.seq_kv[-1] - (m.seq_kv[-2] if len(m.seq_kv) > 1 else 0))
+    assert m.pre_tokens == lk
+    assert bench.visible_pairs(m) == bench.visible_pairs(W.SparseModeInput(**{**m.fields(), "pre_tokens": lk + 999}))
+    assert bench.visible_pairs(diag) < bench.visible_pairs(m)
+
+
+def test_varlen_prefill_problem_is_rectangular():
+    p = W.make_problem("varlen_prefill16k", N=2048, Hq=4, Hkv=2)
+    assert p.q.shape[2] == p.mask.Nq and p.k.shape[2] == p.v.shape[2] == p.mask.Nk == 2048
