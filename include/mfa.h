@@ -1,7 +1,8 @@
 /*
- * mfa.h -- mask-aware flash-attention forward pass for NVIDIA B200 (sm_100a).
+ * mfa.h -- mask-aware flash attention (forward pass and gradients) for NVIDIA
+ * B200 (sm_100a).
  *
- * C ABI of libmfa.so. Two calls carry the computation:
+ * C ABI of libmfa.so. Two calls carry the forward computation:
  *
  *   mfa_build_tile_map  reduces a compact mask description to a per-tile
  *                       SKIP / FULL / PARTIAL map plus, for every query tile,
@@ -14,6 +15,8 @@
  *                       natural-log log-sum-exp of every query row, visiting
  *                       only the listed key tiles (FlashMask author response:
  *                       calculations for fully masked blocks are unnecessary).
+ *   mfa_bwd             computes dq, dk, dv through the same map (FlashMask's
+ *                       masks serve training first, per the author response).
  *
  * Conventions shared by every call:
  *
@@ -73,7 +76,7 @@ typedef enum { MFA_MASK_COLWISE = 0, MFA_MASK_BAND = 1, MFA_MASK_BLOCKSEL = 2 } 
 /* Device error word bits (mfa_tile_map.err). */
 #define MFA_DEVERR_BOUNDS 1u   /* a column bound outside [0, Nq]                      */
 #define MFA_DEVERR_SEL 2u      /* a selection entry outside [-1, ceil(Nk/64))         */
-#define MFA_DEVERR_TIMEOUT 4u  /* a bounded wait in mfa_fwd gave up; outputs invalid  */
+#define MFA_DEVERR_TIMEOUT 4u  /* a bounded wait in mfa_fwd / mfa_bwd gave up; outputs invalid */
 #define MFA_DEVERR_MAP 8u      /* mfa_fwd read a tile list entry outside [0, nkt)     */
 
 /* A 4-D tensor [B, H, N, D]; strides in ELEMENTS, stride[3] must be 1. */
@@ -257,6 +260,42 @@ mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v
 mfa_status mfa_fwd_noalloc(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v,
                            const mfa_mask_desc* mask, int32_t block_q, int32_t block_k,
                            const mfa_tensor* out, float* lse, uint32_t* dev_err, void* stream);
+
+/* Bytes of the DEVICE workspace mfa_bwd needs for these shapes (0 on invalid
+ * shapes). Host only. */
+size_t mfa_bwd_workspace_bytes(int32_t B, int32_t Hq, int32_t Nq, int32_t Nk, int32_t D);
+
+/* Gradients of the forward pass on `stream`, for a loss whose gradient with
+ * respect to out is dout and which does not use lse. This is the derivative
+ * of mfa_fwd's definition by the chain rule; the pages give no backward
+ * formulas. With P = exp(S - lse) on visible pairs and 0 elsewhere:
+ *   dv = P^T dout, dS = P * (dout v^T - rowsum(dout * out)),
+ *   dq = dS k / sqrt(D), dk = dS^T q / sqrt(D).
+ * Key/value head g receives the sums over its query heads g*G .. g*G+G-1.
+ *   q, out, dout, dq  [B, Hq, Nq, D] bf16;  k, v, dk, dv  [B, Hkv, Nk, D] bf16;
+ *       stride[3] == 1, other strides and base addresses 16-byte aligned.
+ *       out and lse are those mfa_fwd returned for q, k, v and this mask.
+ *   lse   float32 [B, Hq, Nq] contiguous.
+ *   mask  description with mask->map built from it by mfa_build_tile_map
+ *         (the forward pass's map serves) with block_k = 128 and block_q 64
+ *         or 128; Hm must be 1. The gradient kernel walks 64-query tiles; a
+ *         128-row map tile gives both of its halves its class.
+ *   workspace  DEVICE buffer of at least mfa_bwd_workspace_bytes(B, Hq, Nq,
+ *         Nk, D) bytes, 256-byte aligned, owned by the caller; no contents are
+ *         needed on entry (it holds an fp32 dq accumulator, per-row softmax
+ *         statistics and the map transposed to per-key-tile lists).
+ * D must be 128. Keys that no query sees get dk = dv = 0. Four kernel
+ * launches: statistics, transposed lists, the gradient kernel, dq conversion
+ * (none of them allocates). A bounded wait that gives up sets
+ * MFA_DEVERR_TIMEOUT in the map's error word. Calls that share a workspace
+ * must not overlap on the GPU.
+ * Errors: MFA_ERR_INVALID_ARG (NULL pointers, small or misaligned workspace),
+ * MFA_ERR_SHAPE_MISMATCH, MFA_ERR_UNSUPPORTED (dtype other than bf16, D != 128,
+ * Hm != 1, block_k != 128), MFA_ERR_CUDA. */
+mfa_status mfa_bwd(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v, const mfa_tensor* out,
+                   const mfa_tensor* dout, const float* lse, const mfa_mask_desc* mask, const mfa_tensor* dq,
+                   const mfa_tensor* dk, const mfa_tensor* dv, void* workspace, size_t workspace_bytes,
+                   void* stream);
 
 /* Synchronise `stream`, read the map's error word into *err_bits (if not
  * NULL) and return MFA_ERR_DEVICE when it is non-zero, MFA_OK otherwise. */

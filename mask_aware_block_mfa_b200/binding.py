@@ -24,7 +24,7 @@ DEVERR_BOUNDS, DEVERR_SEL, DEVERR_TIMEOUT, DEVERR_MAP = 1, 2, 4, 8
 
 EXPORTS = ("mfa_abi_version", "mfa_status_string", "mfa_tile_map_bytes", "mfa_tile_map_init",
            "mfa_build_tile_map", "mfa_fwd", "mfa_fwd_noalloc", "mfa_get_device_status",
-           "mfa_mask_from_sparse_mode")
+           "mfa_mask_from_sparse_mode", "mfa_bwd_workspace_bytes", "mfa_bwd")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -98,6 +98,11 @@ def load(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.mfa_mask_from_sparse_mode.restype = ctypes.c_int
     lib.mfa_mask_from_sparse_mode.argtypes = [ctypes.POINTER(MfaSparseMode)] + [ctypes.c_int32] * 3 + \
         [ctypes.c_void_p] * 4 + [ctypes.POINTER(MfaMaskDesc), ctypes.c_void_p]
+    lib.mfa_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.mfa_bwd_workspace_bytes.argtypes = [ctypes.c_int32] * 5
+    lib.mfa_bwd.restype = ctypes.c_int
+    lib.mfa_bwd.argtypes = [ctypes.POINTER(MfaTensor)] * 5 + [ctypes.c_void_p, ctypes.POINTER(MfaMaskDesc)] + \
+        [ctypes.POINTER(MfaTensor)] * 3 + [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
     if lib.mfa_abi_version() != 1:
         raise RuntimeError("libmfa.so ABI version mismatch")
     _lib = lib
@@ -259,6 +264,25 @@ def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: Device
                                                      lse.data_ptr(), err_ptr, _stream_ptr(stream)))
 
 
+def bwd_workspace_bytes(B: int, Hq: int, Nq: int, Nk: int, D: int) -> int:
+    return int(load().mfa_bwd_workspace_bytes(B, Hq, Nq, Nk, D))
+
+
+def bwd(q, k, v, out, dout, lse, dmask, tmap: TileMap, dq, dk, dv, workspace: torch.Tensor, stream=None) -> None:
+    """dq, dk, dv <- gradients of attention(q, k, v) under dmask for the output
+    gradient dout (out, lse from the forward pass; the map built with 128-key
+    tiles); workspace is a uint8 device tensor of bwd_workspace_bytes()."""
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor")
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous uint8 tensor")
+    dmask.desc.map = ctypes.pointer(tmap.m)
+    ds = [tensor_desc(t) for t in (q, k, v, out, dout, dq, dk, dv)]
+    _check("mfa_bwd", load().mfa_bwd(*(ctypes.byref(d) for d in ds[:5]), lse.data_ptr(), ctypes.byref(dmask.desc),
+                                     *(ctypes.byref(d) for d in ds[5:]), workspace.data_ptr(), workspace.numel(),
+                                     _stream_ptr(stream)))
+
+
 def device_status(tmap: TileMap, stream=None) -> int:
     """Synchronise and return the map's device error bits (0 = none)."""
     bits = ctypes.c_uint32(0)
@@ -287,3 +311,18 @@ class Attention:
             lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
         fwd(q, k, v, self.dmask, self.tmap, out, lse, stream)
         return out, lse
+
+    def backward(self, q, k, v, out, lse, dout, dq=None, dk=None, dv=None, stream=None):
+        """Gradients for the output gradient dout (the map must use 128-key tiles)."""
+        B_, Hq, Nq, D = q.shape
+        need = bwd_workspace_bytes(B_, Hq, Nq, int(k.shape[2]), D)
+        if need == 0:
+            raise ValueError("invalid shapes for the backward pass")
+        ws = getattr(self, "_bwd_ws", None)
+        if ws is None or ws.numel() < need or ws.device != q.device:
+            ws = self._bwd_ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        bwd(q, k, v, out, dout, lse, self.dmask, self.tmap, dq, dk, dv, ws, stream)
+        return dq, dk, dv

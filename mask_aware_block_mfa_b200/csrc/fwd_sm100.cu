@@ -893,7 +893,7 @@ extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   if ((st = check_tensor(q)) != MFA_OK || (st = check_tensor(k)) != MFA_OK || (st = check_tensor(v)) != MFA_OK ||
       (st = check_tensor(out)) != MFA_OK)
     return st;
-  if (!lse) return MFA_ERR_INVALID_ARG;
+  if (!lse && q->N > 0) return MFA_ERR_INVALID_ARG;  // an empty lse may have no storage
   if ((st = check_mask(mask)) != MFA_OK) return st;
   if (!mask->map) return MFA_ERR_INVALID_ARG;
   const mfa_tile_map* map = mask->map;

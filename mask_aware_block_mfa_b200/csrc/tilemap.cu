@@ -21,6 +21,7 @@
 
 #include "mfa.h"
 #include "mfa_internal.h"
+#include "order.cuh"
 
 namespace mfa {
 namespace {
@@ -139,45 +140,6 @@ __device__ __forceinline__ int block_scan256(bool flag, int* s_warp, int* total)
   return before + in_warp;
 }
 
-// Stable counting sort of the E = B*Hm*nqt q-tiles by count, largest first,
-// by one block. Histogram and bucket offsets in shared memory (s_buf, nkt + 1
-// ints); warp 0 then places the entries 32 at a time in index order, so equal
-// counts keep ascending indices.
-__device__ void order_tiles(const int32_t* __restrict__ count, int E, int nkt, int32_t* __restrict__ order,
-                            int* s_buf) {
-  const int t = threadIdx.x;
-  for (int c = t; c <= nkt; c += blockDim.x) s_buf[c] = 0;
-  __syncthreads();
-  for (int e = t; e < E; e += blockDim.x) atomicAdd(&s_buf[count[e]], 1);
-  __syncthreads();
-  if (t == 0) {  // offsets for descending counts
-    int acc = 0;
-    for (int c = nkt; c >= 0; --c) {
-      const int h = s_buf[c];
-      s_buf[c] = acc;
-      acc += h;
-    }
-  }
-  __syncthreads();
-  if (t < 32) {
-    const int lane = t;
-    for (int base = 0; base < E; base += 32) {
-      const int e = base + lane;
-      const int c = e < E ? count[e] : -1;
-      const unsigned peers = __match_any_sync(0xffffffffu, c);
-      const int rank = __popc(peers & ((1u << lane) - 1u));
-      const int leader = __ffs(peers) - 1;
-      int off = 0;
-      if (c >= 0 && lane == leader) off = s_buf[c];
-      off = __shfl_sync(0xffffffffu, off, leader);
-      if (c >= 0) order[off + rank] = e;
-      __syncwarp();
-      if (c >= 0 && lane == leader) s_buf[c] = off + __popc(peers);
-      __syncwarp();
-    }
-  }
-}
-
 __global__ void __launch_bounds__(256) k_tile_classify(MaskArgs m, int BQ, int BK, int nqt, int nkt,
                                                        const int32_t* __restrict__ kmm,
                                                        uint8_t* __restrict__ cls,
@@ -274,7 +236,7 @@ __global__ void __launch_bounds__(256) k_tile_classify(MaskArgs m, int BQ, int B
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  order_tiles(count, static_cast<int>(gridDim.y) * nqt, nkt, order, s_sel);
+  order_by_count_desc(count, static_cast<int>(gridDim.y) * nqt, nkt, order, s_sel);
   if (t == 0) err[3] = 0;
 }
 

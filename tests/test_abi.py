@@ -185,3 +185,52 @@ def test_build_rejects_bad_arguments_on_host(lib):
     assert lib.mfa_build_tile_map(ctypes.byref(sel), ctypes.byref(m), None) == B.MFA_ERR_UNSUPPORTED
     m.tile_list = None
     assert lib.mfa_build_tile_map(ctypes.byref(d), ctypes.byref(m), None) == B.MFA_ERR_INVALID_ARG
+
+
+def test_bwd_workspace_bytes(lib):
+    n = lib.mfa_bwd_workspace_bytes(1, 8, 1000, 900, 128)
+    # fp32 dq accumulator + lse2/Delta padded to 64-row tiles + transposed lists
+    assert n >= 1 * 8 * 1000 * 128 * 4 + 2 * 8 * 1024 * 4 + 8 * 16 * 4
+    assert n % 256 == 0
+    assert lib.mfa_bwd_workspace_bytes(0, 8, 1000, 900, 128) == 0
+    assert lib.mfa_bwd_workspace_bytes(1, 8, -1, 900, 128) == 0
+
+
+def test_bwd_rejects_bad_arguments_on_host(lib):
+    """Every call here fails validation on the host (the pointers are fake, so
+    nothing may be launched)."""
+    m = _fake_map(lib)
+    q, k, v = _fake_tensor(1, 8, 512, 128), _fake_tensor(1, 2, 512, 128), _fake_tensor(1, 2, 512, 128)
+    o, do, dq = _fake_tensor(1, 8, 512, 128), _fake_tensor(1, 8, 512, 128), _fake_tensor(1, 8, 512, 128)
+    dk, dv = _fake_tensor(1, 2, 512, 128), _fake_tensor(1, 2, 512, 128)
+    d = _fake_mask(m)
+    ws_bytes = lib.mfa_bwd_workspace_bytes(1, 8, 512, 512, 128)
+    ws = 0x7300_0000_0000
+
+    def call(q=q, k=k, v=v, o=o, do=do, lse=0x7200_0000_0000, d=d, dq=dq, dk=dk, dv=dv, ws=ws, nbytes=ws_bytes):
+        return lib.mfa_bwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.byref(o), ctypes.byref(do),
+                           lse, ctypes.byref(d), ctypes.byref(dq), ctypes.byref(dk), ctypes.byref(dv), ws, nbytes,
+                           None)
+
+    assert call(lse=0) == B.MFA_ERR_INVALID_ARG
+    assert call(ws=0) == B.MFA_ERR_INVALID_ARG
+    assert call(nbytes=ws_bytes - 256) == B.MFA_ERR_INVALID_ARG               # workspace too small
+    assert call(ws=ws + 16) == B.MFA_ERR_INVALID_ARG                          # not 256-byte aligned
+    assert call(q=_fake_tensor(1, 8, 512, 128, dtype=B.MFA_F32)) == B.MFA_ERR_UNSUPPORTED
+    assert call(dk=_fake_tensor(1, 2, 256, 128)) == B.MFA_ERR_SHAPE_MISMATCH
+    assert call(do=_fake_tensor(1, 8, 256, 128)) == B.MFA_ERR_SHAPE_MISMATCH
+    assert call(k=_fake_tensor(1, 3, 512, 128), v=_fake_tensor(1, 3, 512, 128), dk=_fake_tensor(1, 3, 512, 128),
+                dv=_fake_tensor(1, 3, 512, 128)) == B.MFA_ERR_SHAPE_MISMATCH     # Hq % Hkv != 0
+    d64 = [_fake_tensor(1, h, 512, 64) for h in (8, 2, 2, 8, 8, 8, 2, 2)]
+    assert call(*d64[:5], d=d, dq=d64[5], dk=d64[6], dv=d64[7]) == B.MFA_ERR_UNSUPPORTED   # head dim 64
+    m64 = _fake_map(lib, bq=64, bk=64)
+    assert call(d=_fake_mask(m64)) == B.MFA_ERR_UNSUPPORTED                    # 64-key map tiles
+    m8 = _fake_map(lib, Hm=8)
+    assert call(d=_fake_mask(m8, Hm=8)) == B.MFA_ERR_UNSUPPORTED               # one mask per head
+    dn = _fake_mask(m)
+    dn.map = None
+    assert call(d=dn) == B.MFA_ERR_INVALID_ARG
+    assert call(d=_fake_mask(m, kind=1)) == B.MFA_ERR_SHAPE_MISMATCH          # map built from another kind
+    bad = _fake_tensor(1, 8, 512, 128)
+    bad.stride[3] = 2
+    assert call(dq=bad) == B.MFA_ERR_UNSUPPORTED
