@@ -207,19 +207,28 @@ def run_reference(args, prob, pairs, d, Hq):
     flops = 4.0 * d * pairs * len(heads) / (1 if prob.mask.Hm == 1 else Hq)
     omask = oracle_mask(prob.mask)
     times = []
+    if args.pass_ == "bwd":
+        from oracle import backward as OB
+        flops *= 2.5
+        dout = bwd_output_gradient(prob)
     for s in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        OA.attention(prob.q, prob.k, prob.v, omask, heads=heads)
+        if args.pass_ == "bwd":
+            OB.attention_backward(prob.q, prob.k, prob.v, omask, dout, heads=heads)
+        else:
+            OA.attention(prob.q, prob.k, prob.v, omask, heads=heads)
         if s >= args.warmup:
             times.append(time.perf_counter() - t0)
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     sec = sum(times) / len(times)
     value = flops / sec / 1e12
     return {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "metric": BWD_METRIC if args.pass_ == "bwd" else METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": args.workload, "sample": f"{len(heads)} of {Hq} query heads, all rows"},
+        "config": {"workload": args.workload, "pass": args.pass_,
+                   "sample": f"{len(heads)} of {Hq} query heads, all rows"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"{len(heads)} of {Hq} query heads, all rows, float64 numpy"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -240,6 +249,148 @@ def cpu_baseline(prob, pairs, d, Hq, heads_n):
             "sample": f"{len(heads)} of {Hq} query heads, all rows, float64 numpy ({sec:.1f} s)"}
 
 
+BWD_METRIC = "effective TFLOP/s of the gradient pass (10 d FLOPs per visible pair and head)"
+
+
+def bwd_output_gradient(prob):
+    """Seeded N(0,1) output gradient in bf16, the shape of q."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(prob.seed + 29)
+    return torch.randn(prob.q.shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
+def run_backward(args, prob, pairs, rank, world, local):
+    """Gradient pass (mfa_bwd: statistics, transposed lists, gradient kernel,
+    dq conversion) on a map and forward outputs computed once beforehand."""
+    import torch.distributed as dist
+    from mask_aware_block_mfa_b200 import binding as B
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    Bsz, Hq, Hkv, N, d = prob.shape
+    if prob.q.dtype != torch.bfloat16:
+        raise SystemExit("the gradient pass takes bf16 workloads")
+    bq = BLOCKS[args.workload][0] if BLOCKS[args.workload][1] == 128 else 64
+    flops = 10.0 * d * pairs * (Hq if prob.mask.Hm == 1 else 1)
+    sparse = isinstance(prob.mask, W.SparseModeInput)
+    dmask = B.SparseModeMask(**prob.mask.fields(), device=dev) if sparse else B.DeviceMask(prob.mask, dev)
+    att = B.Attention(dmask, bq, 128, device=dev)
+    q, k, v = (t.to(dev) for t in (prob.q, prob.k, prob.v))
+    dout = bwd_output_gradient(prob).to(dev)
+    att.build()
+    out, lse = att(q, k, v)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        att.backward(q, k, v, out, lse, dout, dq, dk, dv)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize(dev)
+    if B.device_status(att.tmap, stream) != 0:
+        raise RuntimeError("device error word set during warm-up")
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            step()
+    stream.wait_stream(cap)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        for e0, e1 in evs:
+            flush.fill_(1.0)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        time.sleep(0.2)
+    if world > 1:
+        dist.barrier()
+    if B.device_status(att.tmap, stream) != 0:
+        raise RuntimeError("device error word set during the timed steps")
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    total_ms = sum(ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    achieved = flops / (statistics.mean(ms) * 1e-3) / 1e12
+    burst, sustained, src = peaks()
+
+    # End to end: q, k, v, out, lse, dout host -> device, gradients device -> host.
+    hin = [t.pin_memory() for t in (prob.q, prob.k, prob.v, out.cpu(), lse.cpu(), dout.cpu())]
+    hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+    dins = [q, k, v, out, lse, dout]
+    h2d = sum(t.nbytes for t in hin)
+    d2h = sum(t.nbytes for t in hout)
+    e2e_ms = []
+    for s in range(args.e2e_steps + 1):
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for dst, src_t in zip(dins, hin):
+            dst.copy_(src_t, non_blocking=True)
+        step()
+        for dst, src_t in zip(hout, (dq, dk, dv)):
+            dst.copy_(src_t, non_blocking=True)
+        z.record(stream)
+        torch.cuda.synchronize(dev)
+        if s > 0:
+            e2e_ms.append(a.elapsed_time(z))
+    e2e_value = flops * world / (statistics.mean(e2e_ms) * 1e-3) / 1e12
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    res = {
+        "metric": BWD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "pass": "bwd", "desc": W.WORKLOADS[args.workload], "B": Bsz,
+                   "Hq": Hq, "Hkv": Hkv, "N": N, "Nk": prob.Nk, "d": d, "block_q": 64, "block_k": 128,
+                   "map_block_q": bq, "seed": prob.seed, "visible_pairs": pairs,
+                   "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}",
+                   "launch": "each step replayed as a CUDA graph (the four mfa_bwd kernels)"},
+        "frac_of_peak": {"burst": value / burst, "sustained": value / sustained, "peaks": src},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                     "frac": achieved / burst, "traffic": None,
+                     "peak_kind": f"{src} burst bf16 dense; time of the whole mfa_bwd call"},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms": statistics.mean(e2e_ms)},
+        "gpu_launches": 4 * args.steps,  # statistics, transposed lists, gradient kernel, dq conversion
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        from threadpoolctl import threadpool_info
+        from oracle import backward as OB
+        heads = list(range(min(args.oracle_heads, Hq)))
+        t0 = time.perf_counter()
+        OB.attention_backward(prob.q, prob.k, prob.v, oracle_mask(prob.mask), bwd_output_gradient(prob),
+                              heads=heads)
+        sec = time.perf_counter() - t0
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        res["cpu_baseline"] = {"value": 10.0 * d * pairs * len(heads) / sec / 1e12, "unit": "TFLOP/s",
+                               "cores": threads, "kind": "oracle",
+                               "sample": f"{len(heads)} of {Hq} query heads, all rows, float64 numpy ({sec:.1f} s)"}
+    print(json.dumps(res), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -251,6 +402,8 @@ def main():
     ap.add_argument("--reference-heads", type=int, default=1, help="query heads per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
+                    help="fwd: tile map + forward (the headline); bwd: the gradient pass alone")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -267,6 +420,8 @@ def main():
         if rank == 0:
             print(json.dumps(run_reference(args, prob, pairs, d, Hq)), flush=True)
         return
+    if args.pass_ == "bwd":
+        return run_backward(args, prob, pairs, rank, world, local)
 
     import torch.distributed as dist
     from mask_aware_block_mfa_b200 import binding as B

@@ -20,24 +20,25 @@
 // head, 128-key tile). Its key/value tiles stay in shared memory while the
 // item walks every query head g of the group and every listed 64-query tile
 // (an "iteration"). TMEM (512 columns):
-//   [128b, 128b+64)   S^T = K Q^T of iteration parity b (P^T in bf16 over it,
-//                     then dQ^T = K^T dS^T of the same iteration)
-//   [128b+64, 128b+128) dP^T = V dout^T (dS^T in bf16 over it)
+//   [128b, 128b+64)   S^T = K Q^T of iteration parity b (P^T in bf16 over its
+//                     columns [16, 48), then dQ^T = K^T dS^T of the iteration)
+//   [128b+64, 128b+128) dP^T = V dout^T (dS^T in bf16 over [80, 112))
 //   [256, 384) dV,  [384, 512) dK   (accumulated over the item)
 // Rows of S^T, dP^T, dV, dK are keys (TMEM lane = key); rows of dQ^T are head
-// dimensions. Roles (384 threads):
+// dimensions. Roles (512 threads):
 //   warp 0        TMA producer: K, V once per item; Q, dout and the tile's lse
-//                 and Delta per iteration into a two-stage ring.
+//                 and Delta per iteration into a three-stage ring.
 //   warp 1        TMEM owner and MMA issuer: S^T, dP^T of iteration u + 1 go
 //                 out before dV, dK, dQ^T of iteration u, so the tensor core
 //                 works on one iteration while the key-row warps work on the
 //                 other.
-//   warps 4-7     one key row per thread: P^T = exp2(S^T c - lse2) (0 where
-//                 masked), dS^T = P^T (dP^T - Delta), both to TMEM in bf16 and
-//                 dS^T also to shared memory (the B operand of dQ^T); at the
-//                 end of an item dV and dK to global memory.
-//   warps 8-11    one head dimension per thread: dQ^T from TMEM to a staging
-//                 tile, added into the fp32 accumulator by a TMA reduce.
+//   warps 4-11    two warpgroups, one key row per thread, query columns
+//                 0-31 and 32-63: P^T = exp2(S^T c - lse2) (0 where masked),
+//                 dS^T = P^T (dP^T - Delta), both to TMEM in bf16 and dS^T
+//                 also to shared memory (the B operand of dQ^T); at the end of
+//                 an item one warpgroup writes dV and the other dK.
+//   warps 12-15   one head dimension per thread: dQ^T from TMEM to a staging
+//                 tile, added into the fp32 accumulator by TMA reduces.
 //   warps 2-3     idle.
 // Every wait is bounded; a wait that gives up raises the CTA's abort flag and
 // sets MFA_DEVERR_TIMEOUT in the map's error word.
@@ -59,27 +60,35 @@ namespace {
 constexpr int kBQ = 64;    // queries per tile (the MMA N of S^T, dP^T, dQ^T)
 constexpr int kBK = 128;   // keys per tile (the MMA M)
 constexpr int kD = 128;    // head dimension
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kRing = 4;
+constexpr int kStages = 3;  // Q / dout / lse2 / Delta ring
+constexpr uint32_t kPCol = 16;   // packed P^T inside the S^T columns [0, 64) of a parity block
+constexpr uint32_t kDSCol = 80;  // packed dS^T inside the dP^T columns [64, 128)
 
-// ---- shared-memory layout (bytes from a 1024-aligned base) ----
+// ---- shared-memory layout (bytes from the 1024-aligned dynamic base) ----
 constexpr int kKBytes = kBK * kD * 2;    // 32 KB: two 64-column chunks of 128 rows
 constexpr int kQBytes = kBQ * kD * 2;    // 16 KB: two 64-column chunks of 64 rows
 constexpr int kSK = 0;
 constexpr int kSV = kSK + kKBytes;
-constexpr int kSQ = kSV + kKBytes;                // [2 stages]
-constexpr int kSDO = kSQ + 2 * kQBytes;          // [2 stages]
-constexpr int kSDS = kSDO + 2 * kQBytes;         // dS^T: 128 key rows x 64 queries, SW128
-constexpr int kSStg = kSDS + kBK * kBQ * 2;      // dQ staging: 64 rows x 128 fp32
-constexpr int kSLse = kSStg + kBQ * kD * 4;      // [2 stages][64] lse2, then [2][64] Delta
-constexpr int kSBar = kSLse + 4 * kBQ * 4;
-constexpr int kNumBars = 2 + 2 + 2 + 2 + 2 + 1 + 2 + 2 + 1 + 2 + 1 + 2 * kRing;
+constexpr int kSQ = kSV + kKBytes;                 // [kStages]
+constexpr int kSDO = kSQ + kStages * kQBytes;     // [kStages]
+constexpr int kDSBytes = kBK * kBQ * 2;           // dS^T: 128 key rows x 64 queries, SW128
+constexpr int kSDS = kSDO + kStages * kQBytes;    // [2 buffers]
+constexpr int kStgRows = 32;                      // dQ staging: two halves of 32 rows x 128 fp32
+constexpr int kStgBytes = kStgRows * kD * 4;
+constexpr int kSStg = kSDS + 2 * kDSBytes;        // [2 halves]
+constexpr int kSLse = kSStg + 2 * kStgBytes;      // [kStages][64] lse2, then [kStages][64] Delta
+constexpr int kSBar = kSLse + 2 * kStages * kBQ * 4;
+constexpr int kNumBars = 2 + 2 * kStages + 2 * 6 + 1 + 4 + 1 + 2 * kRing;
 constexpr int kSRing = kSBar + ((kNumBars * 8 + 127) / 128) * 128;
-constexpr int kSMisc = kSRing + kRing * 32;
+constexpr int kMeta = 8;  // per-iteration (query tile, head, class byte) published by the producer
+constexpr int kSMeta = kSRing + kRing * 32;
+constexpr int kSMisc = kSMeta + kMeta * 16;
 constexpr int kSmemBytes = kSMisc + 32;
-constexpr int kSmemAlloc = kSmemBytes + 1024;
-static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
-static_assert(kSDS % 1024 == 0 && kSQ % 1024 == 0 && kSDO % 1024 == 0, "SW128 tiles need 1024-byte alignment");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kSDS % 1024 == 0 && kSQ % 1024 == 0 && kSDO % 1024 == 0 && kDSBytes % 1024 == 0,
+              "SW128 tiles need 1024-byte alignment");
 
 struct BwdParams {
   int32_t B, Hq, Hkv, G, Nq, Nk;
@@ -137,7 +146,7 @@ __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const 
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -155,9 +164,10 @@ __device__ __forceinline__ void decode(const BwdParams& p, int w, BwdItem& it) {
 
 // ------------------------------------------------------------------------
 // (1) prep: Delta_i = dout_i . out_i and lse2_i = lse_i log2(e) per query
-// row, padded to nqp = nqt * 64 rows per head (padding and rows without a
+// row, padded to nqp = nq64 * 64 rows per head (padding and rows without a
 // visible key get lse2 = +inf, so their P is exactly 0); dQ accumulator rows
-// zeroed. One warp per row; lane l handles head dimensions 4l .. 4l + 3.
+// zeroed. Half a warp per row: lane l of the half handles head dimensions
+// 8l .. 8l + 7 with 16-byte loads.
 // ------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_bwd_prep(const __nv_bfloat16* __restrict__ out, int64_t os0, int64_t os1,
                                                   int64_t os2, const __nv_bfloat16* __restrict__ dout, int64_t ds0,
@@ -165,29 +175,34 @@ __global__ void __launch_bounds__(256) k_bwd_prep(const __nv_bfloat16* __restric
                                                   int Nq, int nqp, int64_t rows, float* __restrict__ lse2,
                                                   float* __restrict__ delta, float* __restrict__ dq_acc,
                                                   uint32_t* __restrict__ words) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int hl = threadIdx.x & 15;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 4) + (threadIdx.x >> 4);
   if (blockIdx.x == 0 && threadIdx.x < 4) words[threadIdx.x] = 0u;
-  if (row >= rows) return;
+  if (row >= rows) return;  // whole half-warps leave together (rows are per half-warp)
   const int64_t bh = row / nqp;
   const int i = static_cast<int>(row % nqp);
   const int b = static_cast<int>(bh / Hq), h = static_cast<int>(bh % Hq);
   float dl = 0.f, l2 = INFINITY;
+  const unsigned half_mask = (threadIdx.x & 16) ? 0xffff0000u : 0x0000ffffu;
   if (i < Nq) {
-    const uint2 o = *reinterpret_cast<const uint2*>(out + b * os0 + h * os1 + i * os2 + 4 * lane);
-    const uint2 g = *reinterpret_cast<const uint2*>(dout + b * ds0 + h * ds1 + i * ds2 + 4 * lane);
-    const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.x));
-    const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.y));
-    const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g.x));
-    const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&g.y));
-    dl = o0.x * g0.x + o0.y * g0.y + o1.x * g1.x + o1.y * g1.y;
+    const uint4 o = *reinterpret_cast<const uint4*>(out + b * os0 + h * os1 + i * os2 + 8 * hl);
+    const uint4 g = *reinterpret_cast<const uint4*>(dout + b * ds0 + h * ds1 + i * ds2 + 8 * hl);
+    const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
-    for (int d = 16; d > 0; d >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, d);
+    for (int c = 0; c < 4; ++c) {
+      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[c]));
+      const float2 z = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gw[c]));
+      dl = fmaf(a.x, z.x, fmaf(a.y, z.y, dl));
+    }
+#pragma unroll
+    for (int d = 8; d > 0; d >>= 1) dl += __shfl_xor_sync(half_mask, dl, d);
     const float l = lse[bh * Nq + i];
     l2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
-    reinterpret_cast<float4*>(dq_acc + (bh * Nq + i) * kD)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4* acc = reinterpret_cast<float4*>(dq_acc + (bh * Nq + i) * kD);
+    acc[2 * hl] = make_float4(0.f, 0.f, 0.f, 0.f);
+    acc[2 * hl + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  if (lane == 0) {
+  if (hl == 0) {
     lse2[row] = l2;
     delta[row] = dl;
   }
@@ -262,32 +277,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ lse2,
                    const float* __restrict__ delta, const BwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // The SW128 operand tiles need a 1024-byte aligned base; the declaration
+  // asks for it and this checks it (uniformly, before any barrier exists).
+  if ((smem_u32(smem) & 1023u) != 0u) {
+    if (threadIdx.x == 0) atomicOr(p.err, MFA_DEVERR_TIMEOUT);
+    return;
+  }
   uint8_t* sK = smem + kSK;
   uint8_t* sV = smem + kSV;
   uint8_t* sQ = smem + kSQ;
   uint8_t* sDO = smem + kSDO;
   uint8_t* sDS = smem + kSDS;
-  float* sStg = reinterpret_cast<float*>(smem + kSStg);
-  float* sLse = reinterpret_cast<float*>(smem + kSLse);      // [2][64]
-  float* sDelta = sLse + 2 * kBQ;                             // [2][64]
+  float* sStg = reinterpret_cast<float*>(smem + kSStg);       // [2][32][128]
+  float* sLse = reinterpret_cast<float*>(smem + kSLse);       // [kStages][64]
+  float* sDelta = sLse + kStages * kBQ;                       // [kStages][64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSBar);
-  uint64_t* kv_full = bars;           // 1
-  uint64_t* kv_empty = kv_full + 1;   // 1
-  uint64_t* q_full = kv_empty + 1;    // [2]
-  uint64_t* q_empty = q_full + 2;     // [2]
-  uint64_t* s_full = q_empty + 2;     // [2]
-  uint64_t* p_full = s_full + 2;      // [2]
-  uint64_t* ds_free = p_full + 2;     // 1
-  uint64_t* dq_full = ds_free + 1;    // [2]
-  uint64_t* dq_free = dq_full + 2;    // [2]
-  uint64_t* kv_done = dq_free + 2;    // 1
-  uint64_t* stg = kv_done + 1;        // [0] full, [1] free
-  uint64_t* drain = stg + 2;          // 1
-  uint64_t* sched_full = drain + 1;   // [kRing]
+  uint64_t* kv_full = bars;                  // 1
+  uint64_t* kv_empty = kv_full + 1;          // 1
+  uint64_t* q_full = kv_empty + 1;           // [kStages]
+  uint64_t* q_empty = q_full + kStages;      // [kStages]
+  uint64_t* s_full = q_empty + kStages;      // [2] S^T, dP^T of parity b ready
+  uint64_t* p_full = s_full + 2;             // [2] P^T, dS^T of parity b written
+  uint64_t* ds_free = p_full + 2;            // [2] dS^T buffer b read by its dQ^T MMA
+  uint64_t* dq_full = ds_free + 2;           // [2] dQ^T of parity b ready
+  uint64_t* dq_free = dq_full + 2;           // [2] dQ^T of parity b read out
+  uint64_t* kv_done = dq_free + 4;           // 1   (two spare slots above)
+  uint64_t* stg_full = kv_done + 1;          // [2] staging half written
+  uint64_t* stg_free = stg_full + 2;         // [2] staging half read by its reduce
+  uint64_t* drain = stg_free + 2;            // 1
+  uint64_t* sched_full = drain + 1;          // [kRing]
   uint64_t* sched_empty = sched_full + kRing;
   BwdItem* ring = reinterpret_cast<BwdItem*>(smem + kSRing);
+  int4* meta = reinterpret_cast<int4*>(smem + kSMeta);  // [kMeta] {qt, head, class byte, 0}
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kSMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kSMisc + 4);
 
@@ -297,22 +319,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&p_full[s], 256);  // both key-row warpgroups
+      mbar_init(&ds_free[s], 1);
       mbar_init(&dq_full[s], 1);
       mbar_init(&dq_free[s], 128);
+      mbar_init(&stg_full[s], 128);
+      mbar_init(&stg_free[s], 1);
     }
-    mbar_init(ds_free, 1);
     mbar_init(kv_done, 1);
-    mbar_init(&stg[0], 128);
-    mbar_init(&stg[1], 1);
     mbar_init(drain, 1);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sched_full[i], 1);
-      mbar_init(&sched_empty[i], 1 + 4 + 4);  // the MMA warp and one lane of each key-row and dQ warp
+      mbar_init(&sched_empty[i], 1 + 4 + 4 + 4);  // the MMA warp and one lane of every other consumer warp
     }
     *s_abort = 0;
     fence_mbarrier_init();
@@ -357,12 +381,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++kv_loads;
         const int32_t* lst = p.tlist + static_cast<size_t>(info.e) * p.nq64;
+        const uint8_t* crow = p.cls + static_cast<size_t>(info.b) * p.nqt * p.nkt + info.kt;
         for (int g = 0; g < p.G && !stop; ++g) {
           const int h = info.hkv * p.G + g;
           for (int i = 0; i < info.n; ++i, ++u) {
             const int qt = lst[i];
-            const uint32_t st = u & 1;
-            if (u >= 2 && !mbar_wait(&q_empty[st], ((u - 2) >> 1) & 1, s_abort)) { stop = true; break; }
+            const int cb = crow[static_cast<size_t>(qt / p.qsub) * p.nkt];
+            const uint32_t st = u % kStages;
+            if (u >= kStages && !mbar_wait(&q_empty[st], ((u - kStages) / kStages) & 1, s_abort)) {
+              stop = true;
+              break;
+            }
+            // Slot u % kMeta was last read for iteration u - kMeta: by the
+            // key-row warps before p_full(u - kMeta) and by the dQ warps before
+            // dq_free(u - kMeta). q_empty(u - kStages), waited for above, needs
+            // the dQ^T MMA of u - 3, whose S^T waited for dq_free(u - 5), which
+            // follows p_full(u - 5); kMeta = 8 > 5.
+            meta[u % kMeta] = make_int4(qt, h, cb, 0);
             mbar_arrive_expect_tx(&q_full[st], 2 * kQBytes + 2 * kBQ * 4);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
@@ -379,7 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Let the copies already issued land before shared memory is released.
         volatile int no_abort = 0;
         if (kv_loads > 0) mbar_wait(kv_full, (kv_loads - 1) & 1, &no_abort);
-        for (uint32_t j = (u > 2 ? u - 2 : 0); j < u; ++j) mbar_wait(&q_full[j & 1], (j >> 1) & 1, &no_abort);
+        for (uint32_t j = (u > kStages ? u - kStages : 0); j < u; ++j)
+          mbar_wait(&q_full[j % kStages], (j / kStages) & 1, &no_abort);
       }
     }
   } else if (warp == 1) {
@@ -390,19 +426,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t k_kmaj = sdesc_sw128_lo(smem_u32(sK), 16);
     const uint32_t v_kmaj = sdesc_sw128_lo(smem_u32(sV), 16);
     const uint32_t k_mn = sdesc_sw128_lo(smem_u32(sK), kBK * 128);       // 64-dim chunks 16 KB apart
-    const uint32_t ds_mn = sdesc_sw128_lo(smem_u32(sDS), kBK * 128);    // one 64-query chunk
+    const uint32_t ds_mn0 = sdesc_sw128_lo(smem_u32(sDS), kBK * 128);   // one 64-query chunk per buffer
     uint32_t u = 0, kv_items = 0;
     bool ok = true;
 
-    // S^T(u) = K Q(u)^T and dP^T(u) = V dout(u)^T into the columns of parity u & 1.
+    // S^T(u) = K Q(u)^T and dP^T(u) = V dout(u)^T into the TMEM columns of parity u & 1.
     auto issue_sdp = [&](uint32_t uu) -> bool {
-      const uint32_t st = uu & 1;
-      if (!warp_all(mbar_wait(&q_full[st], (uu >> 1) & 1, s_abort))) return false;
-      if (uu >= 2 && !warp_all(mbar_wait(&dq_free[st], ((uu - 2) >> 1) & 1, s_abort))) return false;
+      const uint32_t st = uu % kStages, b = uu & 1;
+      if (!warp_all(mbar_wait(&q_full[st], (uu / kStages) & 1, s_abort))) return false;
+      if (uu >= 2 && !warp_all(mbar_wait(&dq_free[b], ((uu - 2) >> 1) & 1, s_abort))) return false;
       tc_fence_after();
       const uint32_t q_kmaj = sdesc_sw128_lo(smem_u32(sQ + st * kQBytes), 16);
       const uint32_t do_kmaj = sdesc_sw128_lo(smem_u32(sDO + st * kQBytes), 16);
-      const uint32_t d_s = tmem + st * 128;
+      const uint32_t d_s = tmem + b * 128;
 #pragma unroll
       for (int kk = 0; kk < kD / 16; ++kk) {
         const uint32_t off = (kk & 3) * 32;
@@ -415,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_ss(d_s + 64, v_kmaj + (((kk >> 2) * (kBK * 128) + off) >> 4),
                 do_kmaj + (((kk >> 2) * (kBQ * 128) + off) >> 4), idesc_s, kk > 0 ? 1u : 0u);
       }
-      umma_commit(&s_full[st]);
+      umma_commit(&s_full[b]);
       return true;
     };
 
@@ -434,29 +470,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = issue_sdp(u))) break;
       for (uint32_t i = 0; i < n_it; ++i, ++u) {
         if (i + 1 < n_it && !(ok = issue_sdp(u + 1))) break;
-        const uint32_t st = u & 1;
-        if (!(ok = warp_all(mbar_wait(&p_full[st], (u >> 1) & 1, s_abort)))) break;
+        const uint32_t st = u % kStages, b = u & 1;
+        if (!(ok = warp_all(mbar_wait(&p_full[b], (u >> 1) & 1, s_abort)))) break;
         tc_fence_after();
-        const uint32_t buf = tmem + st * 128;
+        const uint32_t buf = tmem + b * 128;
         const uint32_t q_mn = sdesc_sw128_lo(smem_u32(sQ + st * kQBytes), kBQ * 128);
         const uint32_t do_mn = sdesc_sw128_lo(smem_u32(sDO + st * kQBytes), kBQ * 128);
         // dV += P^T dout: K = the 64 queries, 16 per MMA (8 TMEM columns of
         // packed bf16 in A, 16 rows of 128 bytes in B).
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk)
-          umma_ts(tmem + 256, buf + kk * 8, do_mn + kk * (16 * 128 / 16), idesc_kv, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + 256, buf + kPCol + kk * 8, do_mn + kk * (16 * 128 / 16), idesc_kv, (i > 0 || kk > 0) ? 1u : 0u);
         // dK += dS^T Q
 #pragma unroll
         for (int kk = 0; kk < kBQ / 16; ++kk)
-          umma_ts(tmem + 384, buf + 64 + kk * 8, q_mn + kk * (16 * 128 / 16), idesc_kv, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + 384, buf + kDSCol + kk * 8, q_mn + kk * (16 * 128 / 16), idesc_kv, (i > 0 || kk > 0) ? 1u : 0u);
         // dQ^T = K^T dS^T over the 128 keys, into the S^T columns of this parity
         // (the dV MMAs above read P^T from them first; MMAs run in issue order).
+        const uint32_t ds_mn = ds_mn0 + b * (kDSBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk)
           umma_ss(buf, k_mn + kk * (16 * 128 / 16), ds_mn + kk * (16 * 128 / 16), idesc_dq, kk > 0 ? 1u : 0u);
-        umma_commit(&dq_full[st]);
+        umma_commit(&dq_full[b]);
         umma_commit(&q_empty[st]);
-        umma_commit(ds_free);
+        umma_commit(&ds_free[b]);
         if (i + 1 == n_it) {
           umma_commit(kv_done);
           umma_commit(kv_empty);
@@ -469,8 +506,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     umma_commit(drain);
     volatile int no_abort = 0;
     mbar_wait(drain, 0, &no_abort);
-  } else if (wg == 1) {
-    // =================== key rows: P^T, dS^T; dV, dK out ===================
+  } else if (wg == 1 || wg == 2) {
+    // ============ key rows: P^T, dS^T for query columns 32 hq .. 32 hq + 31 ============
+    // Two warpgroups share every key row (TMEM lane) and split the 64 query
+    // columns; at the end of an item one writes dV and the other dK.
+    const int hq = wg - 1;
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const MaskArgs& mk = p.mask;
@@ -485,15 +525,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (info.w < 0) break;
       const int j = info.kt * kBK + r;
       const bool key_ok = j < p.Nk;
-      __nv_bfloat16* dk_row = p.dk + info.b * p.dks0 + info.hkv * p.dks1 + static_cast<int64_t>(j) * p.dks2;
-      __nv_bfloat16* dv_row = p.dv + info.b * p.dvs0 + info.hkv * p.dvs1 + static_cast<int64_t>(j) * p.dvs2;
+      __nv_bfloat16* out_row = hq == 0
+          ? p.dv + info.b * p.dvs0 + info.hkv * p.dvs1 + static_cast<int64_t>(j) * p.dvs2
+          : p.dk + info.b * p.dks0 + info.hkv * p.dks1 + static_cast<int64_t>(j) * p.dks2;
       if (info.n == 0) {  // no query sees these keys
         if (key_ok)
 #pragma unroll 1
-          for (int c = 0; c < kD / 8; ++c) {
-            reinterpret_cast<uint4*>(dk_row)[c] = make_uint4(0, 0, 0, 0);
-            reinterpret_cast<uint4*>(dv_row)[c] = make_uint4(0, 0, 0, 0);
-          }
+          for (int c = 0; c < kD / 8; ++c) reinterpret_cast<uint4*>(out_row)[c] = make_uint4(0, 0, 0, 0);
         continue;
       }
       // The key's mask parameters (fixed for the item).
@@ -504,107 +542,106 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (mk.uts) { uts = mk.uts[idx]; ute = mk.ute[idx]; }
       }
       const int half = r >> 6;  // which 64-key half of the tile (block selection bits)
-      const int32_t* lst = p.tlist + static_cast<size_t>(info.e) * p.nq64;
-      const uint8_t* crow = p.cls + static_cast<size_t>(info.b) * p.nqt * p.nkt + info.kt;
-      for (int g = 0; g < p.G && ok; ++g) {
-        for (int i = 0; i < info.n; ++i, ++u) {
-          const int qt = lst[i];
-          const uint32_t cb = crow[static_cast<size_t>(qt / p.qsub) * p.nkt];
-          const int q0 = qt * kBQ;
-          uint64_t vis = ~0ull;
-          if (!key_ok) {
-            vis = 0ull;
-          } else if ((cb & 3u) == 2u) {
-            if (mk.kind == MFA_MASK_COLWISE) {
-              vis = ~(bits64(lts - q0, lte - q0) | bits64(uts - q0, ute - q0));
-            } else if (mk.kind == MFA_MASK_BAND) {
-              vis = bits64(j - mk.nxt - q0, j + mk.pre + 1 - q0);
-            } else {
-              // selection bit of (64-query sub-block of the map tile, 64-key half)
-              vis = ((cb >> (4 + 2 * (qt % p.qsub) + half)) & 1u) ? bits64(j - q0, 64) : 0ull;
-            }
+      const uint32_t n_it = static_cast<uint32_t>(p.G) * info.n;
+      for (uint32_t i = 0; i < n_it; ++i, ++u) {
+        const uint32_t st = u % kStages, b = u & 1;
+        if (!(ok = warp_all(mbar_wait(&q_full[st], (u / kStages) & 1, s_abort)))) break;  // meta, lse2, Delta
+        const int4 mt = meta[u % kMeta];
+        const int qt = mt.x;
+        const uint32_t cb = static_cast<uint32_t>(mt.z);
+        const int q0 = qt * kBQ + 32 * hq;  // first query of this warpgroup's columns
+        uint32_t vis = ~0u;                 // bit c: query q0 + c visible
+        if (!key_ok) {
+          vis = 0u;
+        } else if ((cb & 3u) == 2u) {
+          if (mk.kind == MFA_MASK_COLWISE) {
+            vis = ~static_cast<uint32_t>(bits64(lts - q0, lte - q0) | bits64(uts - q0, ute - q0));
+          } else if (mk.kind == MFA_MASK_BAND) {
+            vis = static_cast<uint32_t>(bits64(j - mk.nxt - q0, j + mk.pre + 1 - q0));
+          } else {
+            // selection bit of (64-query sub-block of the map tile, 64-key half)
+            vis = ((cb >> (4 + 2 * (qt % p.qsub) + half)) & 1u) ? static_cast<uint32_t>(bits64(j - q0, 32)) : 0u;
           }
-          const uint32_t st = u & 1;
-          if (!(ok = warp_all(mbar_wait(&s_full[st], (u >> 1) & 1, s_abort)))) break;
-          if (!(ok = warp_all(mbar_wait(&q_full[st], (u >> 1) & 1, s_abort)))) break;  // lse2 / Delta landed
-          if (u >= 1 && !(ok = warp_all(mbar_wait(ds_free, (u - 1) & 1, s_abort)))) break;
-          tc_fence_after();
-          const uint32_t tb = tmem + lane_off + st * 128;
-          const float* l2 = sLse + st * kBQ;
-          const float* dl = sDelta + st * kBQ;
-          uint8_t* ds_row = sDS + r * 128;
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t sv[32], dpv[32];
-            tmem_ld_32x32b_x32(tb + h2 * 32, sv);
-            tmem_ld_32x32b_x32(tb + 64 + h2 * 32, dpv);
-            tmem_ld_wait();
-            uint32_t pk[16], dk16[16];
-#pragma unroll
-            for (int c2 = 0; c2 < 16; ++c2) {
-              float pv[2], dsv[2];
-#pragma unroll
-              for (int e2 = 0; e2 < 2; ++e2) {
-                const int c = h2 * 32 + 2 * c2 + e2;
-                const float x = fmaf(__uint_as_float(sv[2 * c2 + e2]), p.scale_log2, -l2[c]);
-                const float pe = ((vis >> c) & 1ull) ? ex2_approx(x) : 0.f;
-                pv[e2] = pe;
-                dsv[e2] = pe * (__uint_as_float(dpv[2 * c2 + e2]) - dl[c]);
-              }
-              pk[c2] = pack_bf16x2(pv[0], pv[1]);
-              dk16[c2] = pack_bf16x2(dsv[0], dsv[1]);
-            }
-            tmem_st_32x32b_x16(tb + h2 * 16, pk);
-            tmem_st_32x32b_x16(tb + 64 + h2 * 16, dk16);
-            // dS^T row r, queries 32 h2 .. 32 h2 + 31 = 16-byte chunks 4 h2 .. 4 h2 + 3,
-            // placed by the 128-byte swizzle (chunk c of row r at c ^ (r & 7)).
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              const int ch = 4 * h2 + c4;
-              *reinterpret_cast<uint4*>(ds_row + ((ch ^ (r & 7)) << 4)) =
-                  make_uint4(dk16[4 * c4], dk16[4 * c4 + 1], dk16[4 * c4 + 2], dk16[4 * c4 + 3]);
-            }
-          }
-          tmem_st_wait();
-          fence_proxy_async_smem();
-          tc_fence_before();
-          mbar_arrive(&p_full[st]);
         }
+        if (!(ok = warp_all(mbar_wait(&s_full[b], (u >> 1) & 1, s_abort)))) break;
+        tc_fence_after();
+        const uint32_t tb = tmem + lane_off + b * 128;
+        uint32_t sv[32], dpv[32];
+        tmem_ld_32x32b_x32(tb + 32 * hq, sv);
+        tmem_ld_32x32b_x32(tb + 64 + 32 * hq, dpv);
+        tmem_ld_wait();
+        const float* l2 = sLse + st * kBQ + 32 * hq;
+        const float* dl = sDelta + st * kBQ + 32 * hq;
+        uint32_t pk[16], dsk[16];
+#pragma unroll
+        for (int c2 = 0; c2 < 16; ++c2) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int c = 2 * c2 + e2;
+            const float x = fmaf(__uint_as_float(sv[c]), p.scale_log2, -l2[c]);
+            const float pe = ((vis >> c) & 1u) ? ex2_approx(x) : 0.f;
+            pv[e2] = pe;
+            dsv[e2] = pe * (__uint_as_float(dpv[c]) - dl[c]);
+          }
+          pk[c2] = pack_bf16x2(pv[0], pv[1]);
+          dsk[c2] = pack_bf16x2(dsv[0], dsv[1]);
+        }
+        // Packed P^T sits at columns [16, 48) and dS^T at [80, 112) of the
+        // parity's block: each warpgroup writes its 16 columns inside the 32 it
+        // alone has just read, so neither overwrites scores the other still reads.
+        tmem_st_32x32b_x16(tb + kPCol + 16 * hq, pk);
+        tmem_st_32x32b_x16(tb + kDSCol + 16 * hq, dsk);
+        // dS^T buffer b was last read by the dQ^T MMA of iteration u - 2.
+        if (u >= 2 && !(ok = warp_all(mbar_wait(&ds_free[b], ((u - 2) >> 1) & 1, s_abort)))) break;
+        // Row r, queries 32 hq .. 32 hq + 31 = 16-byte chunks 4 hq .. 4 hq + 3,
+        // placed by the 128-byte swizzle (chunk c of row r at c ^ (r & 7)).
+        uint8_t* ds_row = sDS + b * kDSBytes + r * 128;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int ch = 4 * hq + c4;
+          *reinterpret_cast<uint4*>(ds_row + ((ch ^ (r & 7)) << 4)) =
+              make_uint4(dsk[4 * c4], dsk[4 * c4 + 1], dsk[4 * c4 + 2], dsk[4 * c4 + 3]);
+        }
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&p_full[b]);
       }
       if (!ok) break;
-      // ---- item epilogue: dV and dK rows of this key ----
+      // ---- item epilogue: dV (hq = 0) or dK (hq = 1) row of this key ----
       if (!(ok = warp_all(mbar_wait(kv_done, items_done & 1, s_abort)))) break;
       ++items_done;
       tc_fence_after();
+      const uint32_t col = hq == 0 ? 256u : 384u;
+      const float sc = hq == 0 ? 1.f : p.scale;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which == 0 ? 256u : 384u;
-        const float sc = which == 0 ? 1.f : p.scale;
-        __nv_bfloat16* row = which == 0 ? dv_row : dk_row;
-#pragma unroll 1
-        for (int c = 0; c < kD / 32; ++c) {
-          uint32_t a[32];
-          tmem_ld_32x32b_x32(tmem + lane_off + col + c * 32, a);
-          tmem_ld_wait();
-          if (key_ok) {
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t a[32];
+        tmem_ld_32x32b_x32(tmem + lane_off + col + c * 32, a);
+        tmem_ld_wait();
+        if (key_ok) {
 #pragma unroll
-            for (int g4 = 0; g4 < 4; ++g4)
-              reinterpret_cast<uint4*>(row)[c * 4 + g4] =
-                  make_uint4(pack_bf16x2(__uint_as_float(a[8 * g4]) * sc, __uint_as_float(a[8 * g4 + 1]) * sc),
-                             pack_bf16x2(__uint_as_float(a[8 * g4 + 2]) * sc, __uint_as_float(a[8 * g4 + 3]) * sc),
-                             pack_bf16x2(__uint_as_float(a[8 * g4 + 4]) * sc, __uint_as_float(a[8 * g4 + 5]) * sc),
-                             pack_bf16x2(__uint_as_float(a[8 * g4 + 6]) * sc, __uint_as_float(a[8 * g4 + 7]) * sc));
-          }
+          for (int g4 = 0; g4 < 4; ++g4)
+            reinterpret_cast<uint4*>(out_row)[c * 4 + g4] =
+                make_uint4(pack_bf16x2(__uint_as_float(a[8 * g4]) * sc, __uint_as_float(a[8 * g4 + 1]) * sc),
+                           pack_bf16x2(__uint_as_float(a[8 * g4 + 2]) * sc, __uint_as_float(a[8 * g4 + 3]) * sc),
+                           pack_bf16x2(__uint_as_float(a[8 * g4 + 4]) * sc, __uint_as_float(a[8 * g4 + 5]) * sc),
+                           pack_bf16x2(__uint_as_float(a[8 * g4 + 6]) * sc, __uint_as_float(a[8 * g4 + 7]) * sc));
         }
       }
       tc_fence_before();
     }
     if (!ok && lane == 0) atomicOr(p.err, MFA_DEVERR_TIMEOUT);
-  } else if (wg == 2) {
+  } else if (wg == 3) {
     // =================== dQ: TMEM -> staging -> TMA reduce-add ===================
+    // Staging is two halves of 32 query rows; the reduce of one half reads
+    // shared memory while the other half is written. Reduce groups go out in
+    // the order half 0, half 1, half 0, ...; after issuing group n, thread 0
+    // waits until group n - 1 has been read and frees its half.
     const int t = (warp & 3) * 32 + lane;  // head dimension = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    uint32_t u = 0, n_stg = 0;
+    uint32_t u = 0, n_grp = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
       const int rs = it % kRing;
@@ -613,37 +650,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sched_empty[rs]);
       if (info.w < 0) break;
-      const int32_t* lst = p.tlist + static_cast<size_t>(info.e) * p.nq64;
-      for (int g = 0; g < p.G && ok; ++g) {
-        const int h = info.hkv * p.G + g;
-        for (int i = 0; i < info.n; ++i, ++u) {
-          const int qt = lst[i];
-          const uint32_t st = u & 1;
-          if (!(ok = warp_all(mbar_wait(&dq_full[st], (u >> 1) & 1, s_abort)))) break;
-          tc_fence_after();
-          uint32_t a[64];
-          tmem_ld_32x32b_x32(tmem + lane_off + st * 128, *reinterpret_cast<uint32_t(*)[32]>(a));
-          tmem_ld_32x32b_x32(tmem + lane_off + st * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(a + 32));
-          tmem_ld_wait();
-          tc_fence_before();
-          mbar_arrive(&dq_free[st]);
-          if (n_stg > 0 && !(ok = warp_all(mbar_wait(&stg[1], (n_stg - 1) & 1, s_abort)))) break;
+      const uint32_t n_it = static_cast<uint32_t>(p.G) * info.n;
+      for (uint32_t i = 0; i < n_it && ok; ++i, ++u) {
+        const uint32_t st = u % kStages, b = u & 1;
+        if (!(ok = warp_all(mbar_wait(&dq_full[b], (u >> 1) & 1, s_abort)))) break;
+        tc_fence_after();
+        // Acquire the producer's meta write for u from q_full(u) itself. The
+        // barrier may already be one phase further (iteration u + kStages,
+        // armed after q_empty(u)); that phase has the other parity, so this
+        // returns at once. Two phases further would need q_empty(u + 3), hence
+        // the S^T of u + 3, hence dq_free(u + 1), which comes after this.
+        if (!(ok = warp_all(mbar_wait(&q_full[st], (u / kStages) & 1, s_abort)))) break;
+        const int4 mt = meta[u % kMeta];
+        const int qt = mt.x, h = mt.y;
+        uint32_t a[64];
+        tmem_ld_32x32b_x32(tmem + lane_off + b * 128, *reinterpret_cast<uint32_t(*)[32]>(a));
+        tmem_ld_32x32b_x32(tmem + lane_off + b * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(a + 32));
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&dq_free[b]);
 #pragma unroll
-          for (int c = 0; c < kBQ; ++c) sStg[c * kD + t] = __uint_as_float(a[c]);
+        for (int hf = 0; hf < 2; ++hf) {
+          // Half hf's previous group is n_grp - 2; it was freed after group n_grp - 1 went out.
+          if (n_grp >= 2 && !(ok = warp_all(mbar_wait(&stg_free[hf], ((n_grp - 2) >> 1) & 1, s_abort)))) break;
+          float* dst = sStg + hf * (kStgRows * kD);
+#pragma unroll
+          for (int c = 0; c < kStgRows; ++c) dst[c * kD + t] = __uint_as_float(a[kStgRows * hf + c]);
           fence_proxy_async_smem();
-          mbar_arrive(&stg[0]);
+          mbar_arrive(&stg_full[hf]);
           if (t == 0) {
             // All 128 threads arrive right above, so this wait ends unless a
             // warp has left on an abort; then it gives up after the bound.
-            if (mbar_wait(&stg[0], n_stg & 1, s_abort)) {
-              tma_reduce_add_4d(&tm_dq, sStg, 0, qt * kBQ, h, info.b);
+            if (mbar_wait(&stg_full[hf], (n_grp >> 1) & 1, s_abort)) {
+              tma_reduce_add_4d(&tm_dq, dst, 0, qt * kBQ + kStgRows * hf, h, info.b);
               bulk_commit();
-              bulk_wait_read0();
+              if (n_grp >= 1) {
+                bulk_wait_read1();
+                mbar_arrive(&stg_free[hf ^ 1]);
+              }
             }
-            mbar_arrive(&stg[1]);
           }
-          __syncwarp();  // reconverge before the next warp-collective tcgen05.ld
-          ++n_stg;
+          __syncwarp();  // reconverge before the next warp-collective instruction
+          ++n_grp;
         }
       }
     }
@@ -716,7 +764,7 @@ bool map_bf16(CUtensorMap* map, const mfa_tensor* t, int rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The fp32 dQ accumulator [B, Hq, Nq, D] (contiguous), 64 rows x 128 columns per box, no swizzle.
+// The fp32 dQ accumulator [B, Hq, Nq, D] (contiguous), 32 rows x 128 columns per box, no swizzle.
 bool map_dq(CUtensorMap* map, void* base, int64_t B, int64_t Hq, int64_t Nq) {
   auto fn = encode_fn_bwd();
   if (!fn) return false;
@@ -724,7 +772,7 @@ bool map_dq(CUtensorMap* map, void* base, int64_t B, int64_t Hq, int64_t Nq) {
                         static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(kD) * 4, static_cast<cuuint64_t>(Nq * kD) * 4,
                            static_cast<cuuint64_t>(Hq * Nq * kD) * 4};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(kD), static_cast<cuuint32_t>(kBQ), 1, 1};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(kD), static_cast<cuuint32_t>(kStgRows), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -807,7 +855,7 @@ extern "C" mfa_status mfa_bwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   // (1) prep
   const int64_t rows = q->B * q->H * static_cast<int64_t>(nqp);
   {
-    const int64_t blocks = (rows + 7) / 8;
+    const int64_t blocks = (rows + 15) / 16;
     if (blocks > 0x7fffffff) return MFA_ERR_UNSUPPORTED;
     k_bwd_prep<<<static_cast<unsigned>(blocks > 0 ? blocks : 1), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(out->data), out->stride[0], out->stride[1], out->stride[2],
@@ -855,7 +903,7 @@ extern "C" mfa_status mfa_bwd(const mfa_tensor* q, const mfa_tensor* k, const mf
     p.sched = words;
     static bool attr_set = false;
     if (!attr_set) {
-      if (cudaFuncSetAttribute(mfa_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) !=
+      if (cudaFuncSetAttribute(mfa_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
           cudaSuccess)
         return MFA_ERR_CUDA;
       attr_set = true;
@@ -863,7 +911,7 @@ extern "C" mfa_status mfa_bwd(const mfa_tensor* q, const mfa_tensor* k, const mf
     const int sms = sm_count_bwd();
     if (sms <= 0) return MFA_ERR_CUDA;
     const int grid = p.n_items < sms ? p.n_items : sms;
-    mfa_bwd_kernel<<<grid, kThreads, kSmemAlloc, s>>>(mq, mk, mv, mdo, mdq, lse2, delta, p);
+    mfa_bwd_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, mdo, mdq, lse2, delta, p);
     if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
   }
   // (4) dq
