@@ -299,8 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_empty = q_full + kStages;      // [kStages]
   uint64_t* s_full = q_empty + kStages;      // [2] S^T, dP^T of parity b ready
   uint64_t* p_full = s_full + 2;             // [2] P^T, dS^T of parity b written
-  uint64_t* ds_free = p_full + 2;            // [2] dS^T buffer b read by its dQ^T MMA
-  uint64_t* dq_full = ds_free + 2;           // [2] dQ^T of parity b ready
+  uint64_t* dq_full = p_full + 2 + 2;        // [2] dQ^T of parity b ready (and dS^T buffer b read)
   uint64_t* dq_free = dq_full + 2;           // [2] dQ^T of parity b read out
   uint64_t* kv_done = dq_free + 4;           // 1   (two spare slots above)
   uint64_t* stg_full = kv_done + 1;          // [2] staging half written
@@ -326,7 +325,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 256);  // both key-row warpgroups
-      mbar_init(&ds_free[s], 1);
       mbar_init(&dq_full[s], 1);
       mbar_init(&dq_free[s], 128);
       mbar_init(&stg_full[s], 128);
@@ -491,9 +489,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk)
           umma_ss(buf, k_mn + kk * (16 * 128 / 16), ds_mn + kk * (16 * 128 / 16), idesc_dq, kk > 0 ? 1u : 0u);
-        umma_commit(&dq_full[b]);
+        umma_commit(&dq_full[b]);  // also frees dS^T buffer b
         umma_commit(&q_empty[st]);
-        umma_commit(&ds_free[b]);
         if (i + 1 == n_it) {
           umma_commit(kv_done);
           umma_commit(kv_empty);
@@ -573,27 +570,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* l2 = sLse + st * kBQ + 32 * hq;
         const float* dl = sDelta + st * kBQ + 32 * hq;
         uint32_t pk[16], dsk[16];
+        // P = 0 where masked. Fully visible 32-column blocks (FULL tiles, most
+        // of the work) skip the per-element select.
+        if (vis == ~0u) {
 #pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) {
-          float pv[2], dsv[2];
+          for (int c2 = 0; c2 < 16; ++c2) {
+            float pv[2], dsv[2];
 #pragma unroll
-          for (int e2 = 0; e2 < 2; ++e2) {
-            const int c = 2 * c2 + e2;
-            const float x = fmaf(__uint_as_float(sv[c]), p.scale_log2, -l2[c]);
-            const float pe = ((vis >> c) & 1u) ? ex2_approx(x) : 0.f;
-            pv[e2] = pe;
-            dsv[e2] = pe * (__uint_as_float(dpv[c]) - dl[c]);
+            for (int e2 = 0; e2 < 2; ++e2) {
+              const int c = 2 * c2 + e2;
+              pv[e2] = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, -l2[c]));
+              dsv[e2] = pv[e2] * (__uint_as_float(dpv[c]) - dl[c]);
+            }
+            pk[c2] = pack_bf16x2(pv[0], pv[1]);
+            dsk[c2] = pack_bf16x2(dsv[0], dsv[1]);
           }
-          pk[c2] = pack_bf16x2(pv[0], pv[1]);
-          dsk[c2] = pack_bf16x2(dsv[0], dsv[1]);
+        } else {
+#pragma unroll
+          for (int c2 = 0; c2 < 16; ++c2) {
+            float pv[2], dsv[2];
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+              const int c = 2 * c2 + e2;
+              const float x = fmaf(__uint_as_float(sv[c]), p.scale_log2, -l2[c]);
+              const float pe = ((vis >> c) & 1u) ? ex2_approx(x) : 0.f;
+              pv[e2] = pe;
+              dsv[e2] = pe * (__uint_as_float(dpv[c]) - dl[c]);
+            }
+            pk[c2] = pack_bf16x2(pv[0], pv[1]);
+            dsk[c2] = pack_bf16x2(dsv[0], dsv[1]);
+          }
         }
         // Packed P^T sits at columns [16, 48) and dS^T at [80, 112) of the
         // parity's block: each warpgroup writes its 16 columns inside the 32 it
         // alone has just read, so neither overwrites scores the other still reads.
         tmem_st_32x32b_x16(tb + kPCol + 16 * hq, pk);
         tmem_st_32x32b_x16(tb + kDSCol + 16 * hq, dsk);
-        // dS^T buffer b was last read by the dQ^T MMA of iteration u - 2.
-        if (u >= 2 && !(ok = warp_all(mbar_wait(&ds_free[b], ((u - 2) >> 1) & 1, s_abort)))) break;
+        // dS^T buffer b was last read by the dQ^T MMA of iteration u - 2, whose
+        // completion is dq_full(u - 2).
+        if (u >= 2 && !(ok = warp_all(mbar_wait(&dq_full[b], ((u - 2) >> 1) & 1, s_abort)))) break;
         // Row r, queries 32 hq .. 32 hq + 31 = 16-byte chunks 4 hq .. 4 hq + 3,
         // placed by the 128-byte swizzle (chunk c of row r at c ^ (r & 7)).
         uint8_t* ds_row = sDS + b * kDSBytes + r * 128;
@@ -650,19 +665,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sched_empty[rs]);
       if (info.w < 0) break;
+      // The iteration's query tile comes from the transposed list in global
+      // memory (written by an earlier launch); it is loaded before the
+      // dq_full wait, which hides the load latency.
+      const int32_t* lst = p.tlist + static_cast<size_t>(info.e) * p.nq64;
       const uint32_t n_it = static_cast<uint32_t>(p.G) * info.n;
       for (uint32_t i = 0; i < n_it && ok; ++i, ++u) {
-        const uint32_t st = u % kStages, b = u & 1;
+        const uint32_t b = u & 1;
+        const int g = static_cast<int>(i / static_cast<uint32_t>(info.n));
+        const int qt = lst[i - static_cast<uint32_t>(g) * info.n];
+        const int h = info.hkv * p.G + g;
         if (!(ok = warp_all(mbar_wait(&dq_full[b], (u >> 1) & 1, s_abort)))) break;
         tc_fence_after();
-        // Acquire the producer's meta write for u from q_full(u) itself. The
-        // barrier may already be one phase further (iteration u + kStages,
-        // armed after q_empty(u)); that phase has the other parity, so this
-        // returns at once. Two phases further would need q_empty(u + 3), hence
-        // the S^T of u + 3, hence dq_free(u + 1), which comes after this.
-        if (!(ok = warp_all(mbar_wait(&q_full[st], (u / kStages) & 1, s_abort)))) break;
-        const int4 mt = meta[u % kMeta];
-        const int qt = mt.x, h = mt.y;
         uint32_t a[64];
         tmem_ld_32x32b_x32(tmem + lane_off + b * 128, *reinterpret_cast<uint32_t(*)[32]>(a));
         tmem_ld_32x32b_x32(tmem + lane_off + b * 128 + 32, *reinterpret_cast<uint32_t(*)[32]>(a + 32));
