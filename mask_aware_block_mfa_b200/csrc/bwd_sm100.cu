@@ -101,6 +101,7 @@ struct BwdParams {
   const int32_t* tlist;   // [B][nkt][nq64] ascending non-SKIP 64-row query tiles
   const int32_t* tcount;  // [B][nkt]
   const int32_t* torder;  // [B * nkt] key tiles, longest list first
+  int32_t order_lpt;      // 1: key tiles longest first; 0: ascending
   __nv_bfloat16* dk;
   int64_t dks0, dks1, dks2;
   __nv_bfloat16* dv;
@@ -152,8 +153,11 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Items (batch, key tile, key/value head) go out with the heads of one key
+// tile together, key tiles either longest list first or in ascending order
+// (see order_lpt).
 __device__ __forceinline__ void decode(const BwdParams& p, int w, BwdItem& it) {
-  const int e = p.torder[w / p.Hkv];
+  const int e = p.order_lpt ? p.torder[w / p.Hkv] : w / p.Hkv;
   it.w = w;
   it.hkv = w % p.Hkv;
   it.e = e;
@@ -911,6 +915,15 @@ extern "C" mfa_status mfa_bwd(const mfa_tensor* q, const mfa_tensor* k, const mf
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(q->D)));
     p.mask = mask_args(mask);
     p.cls = map->tile_class; p.tlist = tlist; p.tcount = tcount; p.torder = torder;
+    // Work order. With many items per CTA and a contiguous mask (documents,
+    // bands), ascending key tiles keep the CTAs working at any moment on
+    // neighbouring key tiles, which share their query tiles: Q / dout tiles
+    // and dQ accumulator rows stay in L2 (doc32k: 11 % faster than longest
+    // first, which re-read them from DRAM). With few items per CTA the end of
+    // the launch dominates and longest first balances it (doc8k: 10 % faster);
+    // block-selection lists are scattered, so there only the balance counts.
+    const int sms_ = sm_count_bwd();
+    p.order_lpt = (mask->kind == MFA_MASK_BLOCKSEL || n_items64 < 8 * static_cast<int64_t>(sms_ > 0 ? sms_ : 148)) ? 1 : 0;
     p.dk = static_cast<__nv_bfloat16*>(dk->data); p.dks0 = dk->stride[0]; p.dks1 = dk->stride[1]; p.dks2 = dk->stride[2];
     p.dv = static_cast<__nv_bfloat16*>(dv->data); p.dvs0 = dv->stride[0]; p.dvs1 = dv->stride[1]; p.dvs2 = dv->stride[2];
     p.err = map->err;
