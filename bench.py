@@ -51,23 +51,30 @@ METRIC = "effective TFLOP/s (visible pairs only) and % of B200 bf16 tensor peak"
 # on; a changed kernel reports traffic as null until it is captured again.
 KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/fwd_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh")
 NCU_TRAFFIC = {
-    "doc8k": (135_914_240, "409987e98985fc1f"),
-    "doc32k": (1_020_204_288, "409987e98985fc1f"),
+    "doc8k": (135_656_192, "80823225e4d4639b"),
+    "doc32k": (1_023_853_056, "80823225e4d4639b"),
+}
+# The same for the gradient kernel (mfa_bwd_kernel) of the backward pass.
+BWD_KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/bwd_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh",
+                      "mask_aware_block_mfa_b200/csrc/order.cuh")
+BWD_NCU_TRAFFIC = {
+    "doc8k": (842_567_936, "e45bc9d337ef5356"),
+    "doc32k": (2_108_606_464, "e45bc9d337ef5356"),
 }
 
 
-def kernel_digest() -> str:
+def kernel_digest(sources=KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
     root = os.path.dirname(os.path.abspath(__file__))
-    for rel in KERNEL_SOURCES:
+    for rel in sources:
         with open(os.path.join(root, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str):
-    entry = NCU_TRAFFIC.get(workload)
-    return entry[0] if entry and entry[1] == kernel_digest() else None
+def ncu_traffic(workload: str, table=None, sources=KERNEL_SOURCES):
+    entry = (NCU_TRAFFIC if table is None else table).get(workload)
+    return entry[0] if entry and entry[1] == kernel_digest(sources) else None
 
 
 def peaks():
@@ -369,8 +376,10 @@ def run_backward(args, prob, pairs, rank, world, local):
                    "launch": "each step replayed as a CUDA graph (the four mfa_bwd kernels)"},
         "frac_of_peak": {"burst": value / burst, "sustained": value / sustained, "peaks": src},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
-                     "frac": achieved / burst, "traffic": None,
-                     "peak_kind": f"{src} burst bf16 dense; time of the whole mfa_bwd call"},
+                     "frac": achieved / burst,
+                     "traffic": ncu_traffic(args.workload, BWD_NCU_TRAFFIC, BWD_KERNEL_SOURCES),
+                     "peak_kind": f"{src} burst bf16 dense; achieved over the whole mfa_bwd call, "
+                                  "traffic of its gradient kernel"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms": statistics.mean(e2e_ms)},
         "gpu_launches": 4 * args.steps,  # statistics, transposed lists, gradient kernel, dq conversion

@@ -31,6 +31,12 @@ def test_ncu_traffic_follows_the_kernel_digest():
     for name, (nbytes, dig) in bench.NCU_TRAFFIC.items():
         assert nbytes > 0 and len(dig) == 16
         assert bench.ncu_traffic(name) == (nbytes if dig == digest else None)
+    bwd_digest = bench.kernel_digest(bench.BWD_KERNEL_SOURCES)
+    assert bwd_digest != digest
+    for name, (nbytes, dig) in bench.BWD_NCU_TRAFFIC.items():
+        assert nbytes > 0 and len(dig) == 16
+        got = bench.ncu_traffic(name, bench.BWD_NCU_TRAFFIC, bench.BWD_KERNEL_SOURCES)
+        assert got == (nbytes if dig == bwd_digest else None)
 
 
 @pytest.mark.parametrize("N", [2048, 5000, None])
