@@ -297,6 +297,40 @@ mfa_status mfa_bwd(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v
                    const mfa_tensor* dk, const mfa_tensor* dv, void* workspace, size_t workspace_bytes,
                    void* stream);
 
+/* Bytes of the DEVICE workspace mfa_decode needs with n_split parts per list
+ * (0 = the split mfa_decode chooses; 256 when no workspace is used; 0 on
+ * invalid sizes). Host only. */
+size_t mfa_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t Nq, int32_t D, int32_t sel_k,
+                                  int32_t n_split);
+
+/* Selected-key attention for a few query rows (decode), from the pull request
+ * "vulkan : selected-key flash attention for QSA block selection" (overview
+ * and kernel description), on `stream`.
+ *   q, out  [B, Hq, Nq, D] bf16;  k, v  [B, Hkv, Nk, D] bf16 (the cache);
+ *           D in {128, 256}, G = Hq / Hkv in {1, 2, 4, 8, 16}, G * D <= 2048;
+ *           stride[3] == 1, other strides and base addresses 16-byte aligned.
+ *   sel     DEVICE int32 [B, Hkv, Nq, sel_k] contiguous: for every (batch,
+ *           key/value head, query row) a list of 64-key block indices, shared
+ *           by the head's G query heads. -1 = no entry; a block listed twice
+ *           counts once; entries outside [-1, ceil(Nk/64)) are ignored and set
+ *           MFA_DEVERR_SEL. sel_k <= 256.
+ *   Query row i sits at position i + Nk - Nq: it sees key j when j's block is
+ *   listed and j <= i + Nk - Nq (with Nq == Nk, the rule of MFA_MASK_BLOCKSEL).
+ *   Rows that see no key get out = 0 and lse = -inf.
+ *   lse     float32 [B, Hq, Nq] contiguous, natural log.
+ *   n_split parts per list (0 = chosen for at least two CTAs per SM); with
+ *           n_split > 1 the parts are combined by a second kernel (empty parts
+ *           carry m = -FLT_MAX, so no exp(-inf - -inf) arises) and `workspace`
+ *           (DEVICE, 256-byte aligned, mfa_decode_workspace_bytes bytes, owned
+ *           by the caller) holds the partial results.
+ *   dev_err DEVICE uint32 the kernels OR MFA_DEVERR_* bits into (required; the
+ *           caller clears it).
+ * Errors: MFA_ERR_INVALID_ARG, MFA_ERR_SHAPE_MISMATCH, MFA_ERR_UNSUPPORTED
+ * (dtype, D, G, sizes, Nk == 0), MFA_ERR_CUDA. */
+mfa_status mfa_decode(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v, const int32_t* sel,
+                      int32_t sel_k, const mfa_tensor* out, float* lse, int32_t n_split, void* workspace,
+                      size_t workspace_bytes, uint32_t* dev_err, void* stream);
+
 /* Synchronise `stream`, read the map's error word into *err_bits (if not
  * NULL) and return MFA_ERR_DEVICE when it is non-zero, MFA_OK otherwise. */
 mfa_status mfa_get_device_status(const mfa_tile_map* map, void* stream, uint32_t* err_bits);

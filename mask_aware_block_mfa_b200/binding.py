@@ -24,7 +24,8 @@ DEVERR_BOUNDS, DEVERR_SEL, DEVERR_TIMEOUT, DEVERR_MAP = 1, 2, 4, 8
 
 EXPORTS = ("mfa_abi_version", "mfa_status_string", "mfa_tile_map_bytes", "mfa_tile_map_init",
            "mfa_build_tile_map", "mfa_fwd", "mfa_fwd_noalloc", "mfa_get_device_status",
-           "mfa_mask_from_sparse_mode", "mfa_bwd_workspace_bytes", "mfa_bwd")
+           "mfa_mask_from_sparse_mode", "mfa_bwd_workspace_bytes", "mfa_bwd", "mfa_decode_workspace_bytes",
+           "mfa_decode")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -103,6 +104,13 @@ def load(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.mfa_bwd.restype = ctypes.c_int
     lib.mfa_bwd.argtypes = [ctypes.POINTER(MfaTensor)] * 5 + [ctypes.c_void_p, ctypes.POINTER(MfaMaskDesc)] + \
         [ctypes.POINTER(MfaTensor)] * 3 + [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    lib.mfa_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.mfa_decode_workspace_bytes.argtypes = [ctypes.c_int32] * 7
+    lib.mfa_decode.restype = ctypes.c_int
+    lib.mfa_decode.argtypes = [ctypes.POINTER(MfaTensor)] * 3 + [ctypes.c_void_p, ctypes.c_int32,
+                                                                 ctypes.POINTER(MfaTensor), ctypes.c_void_p,
+                                                                 ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
+                                                                 ctypes.c_void_p, ctypes.c_void_p]
     if lib.mfa_abi_version() != 1:
         raise RuntimeError("libmfa.so ABI version mismatch")
     _lib = lib
@@ -281,6 +289,48 @@ def bwd(q, k, v, out, dout, lse, dmask, tmap: TileMap, dq, dk, dv, workspace: to
     _check("mfa_bwd", load().mfa_bwd(*(ctypes.byref(d) for d in ds[:5]), lse.data_ptr(), ctypes.byref(dmask.desc),
                                      *(ctypes.byref(d) for d in ds[5:]), workspace.data_ptr(), workspace.numel(),
                                      _stream_ptr(stream)))
+
+
+def decode_workspace_bytes(B: int, Hq: int, Hkv: int, Nq: int, D: int, sel_k: int, n_split: int = 0) -> int:
+    return int(load().mfa_decode_workspace_bytes(B, Hq, Hkv, Nq, D, sel_k, n_split))
+
+
+class Decode:
+    """Selected-key attention for a few query rows (mfa_decode): keeps the
+    split-K workspace and the device error word between calls."""
+
+    def __init__(self, n_split: int = 0):
+        self.n_split = n_split
+        self.ws = None
+        self.err = None
+
+    def __call__(self, q, k, v, sel, out=None, lse=None, stream=None):
+        """sel: int32 device tensor [B, Hkv, Nq, sel_k] of 64-key block indices (-1 = none)."""
+        if sel.dtype != torch.int32 or not sel.is_contiguous() or sel.dim() != 4:
+            raise ValueError("sel must be a contiguous int32 [B, Hkv, Nq, sel_k] tensor")
+        B_, Hq, Nq, D = q.shape
+        Hkv = int(k.shape[1])
+        sel_k = int(sel.shape[-1])
+        need = decode_workspace_bytes(B_, Hq, Hkv, Nq, D, sel_k, self.n_split)
+        if need == 0:
+            raise ValueError("invalid decode sizes")
+        if self.ws is None or self.ws.numel() < need or self.ws.device != q.device:
+            self.ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+        if self.err is None or self.err.device != q.device:
+            self.err = torch.zeros(1, dtype=torch.int32, device=q.device)
+        out = torch.empty_like(q) if out is None else out
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if lse is None else lse
+        qd, kd, vd, od = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
+        _check("mfa_decode", load().mfa_decode(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), sel.data_ptr(),
+                                               sel_k, ctypes.byref(od), lse.data_ptr(), self.n_split,
+                                               self.ws.data_ptr(), self.ws.numel(), self.err.data_ptr(),
+                                               _stream_ptr(stream)))
+        return out, lse
+
+    def status(self) -> int:
+        """Synchronise and return the device error bits (0 = none)."""
+        torch.cuda.synchronize()
+        return 0 if self.err is None else int(self.err.item())
 
 
 def device_status(tmap: TileMap, stream=None) -> int:

@@ -340,6 +340,53 @@ def make_problem(name: str, seed: Optional[int] = None, N: Optional[int] = None,
     return Problem(name, q, k, v, mask, seed)
 
 
+# ----------------------------------------------------------------------------
+# Selected-key decode (a few query rows against a long cache)
+# ----------------------------------------------------------------------------
+
+DECODE_WORKLOADS = {
+    "decode_sel64k": "B=8 Hq=32 Hkv=8 (GQA 4) d=256 Nq=1 Nk=65536 bf16; per (batch, K/V head) the top 32 of "
+                     "uniform scores over the 64-key blocks (2048 selected keys)",
+}
+DECODE_SHAPES = {  # name: (B, Hq, Hkv, Nq, Nk, d, sel_k)
+    "decode_sel64k": (8, 32, 8, 1, 65536, 256, 32),
+}
+DECODE_SEEDS = {"decode_sel64k": 7000}
+
+
+def decode_selection(rng: np.random.Generator, B: int, Hkv: int, Nq: int, Nk: int, sel_k: int,
+                     pads: int = 0, dups: int = 0) -> np.ndarray:
+    """int32 [B, Hkv, Nq, sel_k]: per list the top (sel_k - pads - dups) of
+    uniform scores over the 64-key blocks up to the row's position (i + Nk -
+    Nq), then `dups` repeated entries and `pads` entries of -1, shuffled."""
+    nblk = (Nk + 63) // 64
+    out = np.full((B, Hkv, Nq, sel_k), -1, dtype=np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            for i in range(Nq):
+                last = i + Nk - Nq
+                avail = last // 64 + 1 if last >= 0 else 0
+                avail = min(avail, nblk)
+                take = min(sel_k - pads - dups, avail)
+                if take <= 0:
+                    continue
+                picks = np.argsort(rng.random(avail), kind="stable")[:take]
+                row = list(picks)
+                row += list(rng.choice(picks, size=min(dups, len(picks)), replace=True)) if dups else []
+                row += [-1] * (sel_k - len(row))
+                out[b, g, i] = rng.permutation(np.asarray(row, dtype=np.int32))
+    return out
+
+
+def make_decode_problem(name: str):
+    """q, k, v (seeded N(0,1), bf16, on the CPU) and the selection lists of a decode workload."""
+    B, Hq, Hkv, Nq, Nk, d, sel_k = DECODE_SHAPES[name]
+    seed = DECODE_SEEDS[name]
+    q, k, v = randn_qkv(seed + 17, B, Hq, Hkv, Nq, d, torch.bfloat16, Nk=Nk)
+    sel = decode_selection(np.random.default_rng(seed), B, Hkv, Nq, Nk, sel_k)
+    return q, k, v, sel
+
+
 def random_colwise(rng: np.random.Generator, B: int, Hm: int, Nq: int, Nk: int,
                    p_empty: float = 0.3) -> MaskDesc:
     """Arbitrary column bounds in [0, Nq] (empty intervals included) for stress tests."""

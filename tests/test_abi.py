@@ -234,3 +234,38 @@ def test_bwd_rejects_bad_arguments_on_host(lib):
     bad = _fake_tensor(1, 8, 512, 128)
     bad.stride[3] = 2
     assert call(dq=bad) == B.MFA_ERR_UNSUPPORTED
+
+
+def test_decode_rejects_bad_arguments_on_host(lib):
+    """Every call here fails validation on the host (fake pointers: nothing may be launched)."""
+    q, k, v, o = _fake_tensor(1, 8, 1, 256), _fake_tensor(1, 2, 4096, 256), _fake_tensor(1, 2, 4096, 256), \
+        _fake_tensor(1, 8, 1, 256)
+    sel, lse, ws, err = 0x7400_0000_0000, 0x7200_0000_0000, 0x7300_0000_0000, 0x7500_0000_0000
+    need = lib.mfa_decode_workspace_bytes(1, 8, 2, 1, 256, 16, 4)
+    assert need > 256 and need % 256 == 0
+    assert lib.mfa_decode_workspace_bytes(1, 8, 3, 1, 256, 16, 4) == 0          # Hq % Hkv != 0
+
+    def call(q=q, k=k, v=v, sel=sel, sel_k=16, o=o, lse=lse, n_split=4, ws=ws, nbytes=need, err=err):
+        return lib.mfa_decode(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), sel, sel_k, ctypes.byref(o), lse,
+                              n_split, ws, nbytes, err, None)
+
+    assert call(err=0) == B.MFA_ERR_INVALID_ARG
+    assert call(sel=0) == B.MFA_ERR_INVALID_ARG
+    assert call(lse=0) == B.MFA_ERR_INVALID_ARG
+    assert call(sel_k=0) == B.MFA_ERR_INVALID_ARG
+    assert call(n_split=-1) == B.MFA_ERR_INVALID_ARG
+    assert call(nbytes=need - 256) == B.MFA_ERR_INVALID_ARG                   # workspace too small
+    assert call(ws=0) == B.MFA_ERR_INVALID_ARG
+    assert call(sel_k=257) == B.MFA_ERR_UNSUPPORTED
+    d64 = [_fake_tensor(1, h, n, 64) for h, n in ((8, 1), (2, 4096), (2, 4096), (8, 1))]
+    assert call(q=d64[0], k=d64[1], v=d64[2], o=d64[3]) == B.MFA_ERR_UNSUPPORTED   # head dim 64
+    g3 = [_fake_tensor(1, h, n, 256) for h, n in ((6, 1), (2, 4096), (2, 4096), (6, 1))]
+    assert call(q=g3[0], k=g3[1], v=g3[2], o=g3[3]) == B.MFA_ERR_UNSUPPORTED      # G = 3
+    g16 = [_fake_tensor(1, h, n, 256) for h, n in ((32, 1), (2, 4096), (2, 4096), (32, 1))]
+    assert call(q=g16[0], k=g16[1], v=g16[2], o=g16[3]) == B.MFA_ERR_UNSUPPORTED  # G * D > 2048
+    assert call(v=_fake_tensor(1, 2, 2048, 256)) == B.MFA_ERR_SHAPE_MISMATCH
+    assert call(o=_fake_tensor(1, 8, 2, 256)) == B.MFA_ERR_SHAPE_MISMATCH
+    k0, v0 = _fake_tensor(1, 2, 0, 256, addr=0), _fake_tensor(1, 2, 0, 256, addr=0)
+    assert call(k=k0, v=v0) == B.MFA_ERR_UNSUPPORTED                             # no keys
+    f32 = _fake_tensor(1, 8, 1, 256, dtype=B.MFA_F32)
+    assert call(q=f32) == B.MFA_ERR_UNSUPPORTED
