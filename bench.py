@@ -400,25 +400,206 @@ def run_backward(args, prob, pairs, rank, world, local):
     print(json.dumps(res), flush=True)
 
 
+DECODE_METRIC = "GB/s of the selected-key decode (visible selected K/V rows + q + out + lse + lists)"
+
+
+def decode_bytes(q, k, sel):
+    """Algorithmic bytes of one decode call: every visible key of every
+    deduplicated listed block, K and V, once per (batch, key/value head, row)
+    (the G query heads share it), plus q, out, lse and the lists."""
+    B_, Hq, Nq, d = q.shape
+    Nk = int(k.shape[2])
+    keys = 0
+    sel3 = sel.reshape(-1, Nq, sel.shape[-1])
+    for r in range(sel3.shape[0]):
+        for i in range(Nq):
+            last = i + Nk - Nq
+            for blk in set(int(x) for x in sel3[r, i] if x >= 0):
+                keys += max(0, min(64 * blk + 64, last + 1, Nk) - 64 * blk)
+    elem = 2
+    return keys * d * elem * 2 + 2 * B_ * Hq * Nq * d * elem + B_ * Hq * Nq * 4 + sel.size * 4
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def run_decode(args, rank, world, local):
+    """Selected-key decode (mfa_decode and, with several parts per list, its
+    combine kernel) on a cache resident in HBM."""
+    import torch.distributed as dist
+    from threadpoolctl import threadpool_info
+    from mask_aware_block_mfa_b200 import binding as B
+    q, k, v, sel = W.make_decode_problem(args.workload)
+    B_, Hq, Hkv, Nq, Nk, d, sel_k = W.DECODE_SHAPES[args.workload]
+    nbytes = decode_bytes(q, k, sel)
+    if args.impl == "reference":
+        if rank == 0:
+            from oracle import decode as OD
+            bs = list(range(min(args.reference_heads, B_)))  # a sample of the batch
+            frac = len(bs) / B_
+            times = []
+            for st in range(args.warmup + args.steps):
+                t0 = time.perf_counter()
+                OD.decode_attention(q[bs], k[bs], v[bs], sel[bs])
+                if st >= args.warmup:
+                    times.append(time.perf_counter() - t0)
+            sec = sum(times) / len(times)
+            val = nbytes * frac / sec / 1e9
+            threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+            print(json.dumps({
+                "metric": DECODE_METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": args.workload, "pass": "decode", "sample": f"{len(bs)} of {B_} sequences"},
+                "cpu_baseline": {"value": val, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                 "sample": f"{len(bs)} of {B_} sequences, float64 numpy"},
+                "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+                flush=True)
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    seld = torch.from_numpy(sel).to(dev)
+    out = torch.empty_like(qd)
+    lse = torch.empty(qd.shape[:3], dtype=torch.float32, device=dev)
+    dec = B.Decode(0)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        dec(qd, kd, vd, seld, out, lse)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    if dec.status() != 0:
+        raise RuntimeError("device error bits set during warm-up")
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            step()
+    stream.wait_stream(cap)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        for e0, e1 in evs:
+            flush.fill_(1.0)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        time.sleep(0.2)
+    if world > 1:
+        dist.barrier()
+    if dec.status() != 0:
+        raise RuntimeError("device error bits set during the timed steps")
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    total_ms = sum(ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = nbytes * world * args.steps / (total_ms * 1e-3) / 1e9
+    achieved = nbytes / (statistics.mean(ms) * 1e-3) / 1e9
+    peak, src = hbm_peak()
+    # End to end: the cache stays resident (as in serving); each step copies the
+    # queries and lists in and out / lse back.
+    hq, hsel = q.pin_memory(), torch.from_numpy(sel).pin_memory()
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    e2e_ms = []
+    for st in range(args.e2e_steps + 1):
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        qd.copy_(hq, non_blocking=True)
+        seld.copy_(hsel, non_blocking=True)
+        step()
+        ho.copy_(out, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+        z.record(stream)
+        torch.cuda.synchronize(dev)
+        if st > 0:
+            e2e_ms.append(a.elapsed_time(z))
+    e2e_value = nbytes * world / (statistics.mean(e2e_ms) * 1e-3) / 1e9
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    n_split = int(dec.ws.numel() > 256)
+    res = {
+        "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "pass": "decode", "desc": W.DECODE_WORKLOADS[args.workload],
+                   "B": B_, "Hq": Hq, "Hkv": Hkv, "Nq": Nq, "Nk": Nk, "d": d, "sel_k": sel_k,
+                   "algorithmic_bytes": nbytes, "l2": "flushed between timed steps (256 MiB write)",
+                   "parallelism": f"replicas x{world}", "launch": "each step replayed as a CUDA graph"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_kind": f"{src} HBM copy bandwidth"},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": hq.nbytes + hsel.nbytes,
+                "d2h_bytes_per_step": ho.nbytes + hl.nbytes, "ms": statistics.mean(e2e_ms),
+                "note": "cache resident in HBM; queries and lists copied in, out and lse copied back"},
+        "gpu_launches": (2 if n_split else 1) * args.steps,  # decode kernel (+ combine when the lists are split)
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        from oracle import decode as OD
+        t0 = time.perf_counter()
+        OD.decode_attention(q[:1], k[:1], v[:1], sel[:1])
+        sec = time.perf_counter() - t0
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        res["cpu_baseline"] = {"value": nbytes / B_ / sec / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                               "sample": f"1 of {B_} sequences, float64 numpy ({sec:.1f} s)"}
+    print(json.dumps(res), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="doc8k", choices=sorted(BLOCKS))
+    ap.add_argument("--workload", default=None, choices=sorted(BLOCKS) + sorted(W.DECODE_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--oracle-heads", type=int, default=4, help="query heads in the CPU-baseline sample")
     ap.add_argument("--reference-heads", type=int, default=1, help="query heads per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
-                    help="fwd: tile map + forward (the headline); bwd: the gradient pass alone")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "decode"],
+                    help="fwd: tile map + forward (the headline); bwd: the gradient pass alone; "
+                         "decode: selected-key decode (decode workloads)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.pass_ == "decode":
+        args.workload = args.workload or "decode_sel64k"
+        if args.workload not in W.DECODE_WORKLOADS:
+            raise SystemExit("--pass decode takes a decode workload")
+        return run_decode(args, rank, world, local)
+    args.workload = args.workload or "doc8k"
+    if args.workload not in BLOCKS:
+        raise SystemExit("decode workloads run with --pass decode")
 
     prob = W.make_problem(args.workload)
     Bsz, Hq, Hkv, N, d = prob.shape

@@ -45,9 +45,12 @@ namespace mfa {
 namespace {
 
 constexpr int kBlk = 64;       // keys per selection block
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
-constexpr int kKeysPerWarp = kBlk / kWarps;
+constexpr int kCombineThreads = 256;
+// 16 warps when the query rows and outputs fit 128 registers a thread
+// (G * D <= 1024), else 8: more warps hide more of the shared-memory and
+// shuffle latency of the one CTA that fits an SM.
+template <int D, int G>
+constexpr int kWarpsFor = G * D <= 1024 ? 16 : 8;
 
 struct DecParams {
   int32_t B, Hq, Hkv, G, Nq, Nk, nblk, sel_k, n_split;
@@ -67,15 +70,18 @@ template <int D>
 struct DecCfg {
   static constexpr int kDL = D / 32;                 // head dimensions per lane
   static constexpr int kTile = kBlk * D * 2;         // one K (or V) block: D / 64 boxes of 64 rows x 128 B
-  static constexpr int kK = 0;                       // [2 stages]
-  static constexpr int kV = kK + 2 * kTile;          // [2 stages]
-  static constexpr int kS = kV + 2 * kTile;          // scores / P: [16][64] fp32
-  static constexpr int kList = kS + 16 * kBlk * 4;   // deduplicated list [kMaxSelK]
+  static constexpr int kStages = 3;                  // K/V ring: two blocks in flight while one is used
+  static constexpr int kK = 0;                       // [kStages]
+  static constexpr int kV = kK + kStages * kTile;    // [kStages]
+  static constexpr int kS = kV + kStages * kTile;    // scores [16][64] fp32, then P [64][16]
+  static constexpr int kList = kS + 2 * 16 * kBlk * 4;  // deduplicated list [kMaxSelK]
   static constexpr int kMisc = kList + kMaxSelK * 4; // softmax state, counters, barriers
   static constexpr int kBytes = kMisc + 1024;
-  // The final cross-warp sum of the outputs (G * D <= 2048) reuses the K/V ring
-  // and the score and list space after it, none of which the epilogue reads.
-  static_assert(kWarps * 32 * (2048 / D * kDL + 1) * 4 <= kMisc, "output reduction space");
+  // The final cross-warp sum of the outputs reuses the K/V ring and the score
+  // and list space after it, none of which the epilogue reads: 16 warps with
+  // G * D <= 1024 or 8 warps with G * D <= 2048.
+  static_assert(16 * 32 * (1024 / D * kDL + 1) * 4 <= kMisc, "output reduction space (16 warps)");
+  static_assert(8 * 32 * (2048 / D * kDL + 1) * 4 <= kMisc, "output reduction space (8 warps)");
 };
 
 // Element offset of head dimensions [c0, c0 + n) of key row r in a K/V block
@@ -86,27 +92,21 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c0) {
   return static_cast<uint32_t>(box * (kBlk * 128) + r * 128 + ((ch ^ (r & 7)) << 4) + (c0 & 7) * 2);
 }
 
+// A bf16 pair widened to a packed float pair: bf16 is the upper half of a float.
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Head dimensions [DL lane, DL lane + DL) of key row r as DL / 2 packed pairs.
 template <int DL>
-__device__ __forceinline__ void load_row(const uint8_t* tile, int r, int lane, float (&x)[DL]) {
+__device__ __forceinline__ void load_row2(const uint8_t* tile, int r, int lane, uint64_t (&x)[DL / 2]) {
   const uint8_t* p = tile + sw_off(r, lane * DL);
   if constexpr (DL == 8) {
     const uint4 w = *reinterpret_cast<const uint4*>(p);
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ww[e]));
-      x[2 * e] = f.x;
-      x[2 * e + 1] = f.y;
-    }
+    x[0] = bf2_to_f2(w.x); x[1] = bf2_to_f2(w.y); x[2] = bf2_to_f2(w.z); x[3] = bf2_to_f2(w.w);
   } else {
     const uint2 w = *reinterpret_cast<const uint2*>(p);
-    const uint32_t ww[2] = {w.x, w.y};
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ww[e]));
-      x[2 * e] = f.x;
-      x[2 * e + 1] = f.y;
-    }
+    x[0] = bf2_to_f2(w.x); x[1] = bf2_to_f2(w.y);
   }
 }
 
@@ -150,33 +150,37 @@ __device__ __forceinline__ int row_of_lane(int lane) {
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kWarpsFor<D, G> * 32, 1)
     mfa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const DecParams p) {
   using C = DecCfg<D>;
   constexpr int DL = C::kDL;
+  constexpr int kWarps = kWarpsFor<D, G>;
+  constexpr int kThreads = kWarps * 32;
+  constexpr int kKeysPerWarp = kBlk / kWarps;
+  constexpr int GP = (G + 3) / 4 * 4;  // P row stride (float4 loads)
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = blockIdx.x, i = blockIdx.y;
   const int bg = blockIdx.z, b = bg / p.Hkv, g = bg % p.Hkv;
   const size_t row_unit = (static_cast<size_t>(bg) * p.Nq + i);
 
-  float* sS = reinterpret_cast<float*>(smem + C::kS);          // [G][64] scores, then P
+  float* sS = reinterpret_cast<float*>(smem + C::kS);          // [G][64] scores
+  float* sPT = sS + 16 * kBlk;                                 // [64][GP] P, key-major
   int* sList = reinterpret_cast<int*>(smem + C::kList);
   float* sM = reinterpret_cast<float*>(smem + C::kMisc);       // [16] running max (log2 units)
   float* sL = sM + 16;                                         // [16] running sum
   float* sA = sL + 16;                                         // [16] rescale factor of this block
-  int* sCnt = reinterpret_cast<int*>(sA + 16);                 // [kWarps] list compaction, [8] total
-  volatile int* sFlag = reinterpret_cast<volatile int*>(sCnt + 12);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kMisc + 512);  // [2]
+  int* sCnt = reinterpret_cast<int*>(sA + 16);                 // [kWarps] list compaction, [16] total
+  volatile int* sFlag = reinterpret_cast<volatile int*>(sCnt + 20);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kMisc + 512);  // [kStages]
 
   if ((smem_u32(smem) & 1023u) != 0u) {  // SW128 boxes need a 1024-aligned base (uniform check)
     if (threadIdx.x == 0) atomicOr(p.err, MFA_DEVERR_TIMEOUT);
     return;
   }
   if (threadIdx.x == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
+    for (int st = 0; st < C::kStages; ++st) mbar_init(&full[st], 1);
     *sFlag = 0;
     fence_mbarrier_init();
   }
@@ -192,7 +196,7 @@ __global__ void __launch_bounds__(kThreads)
   for (int e = threadIdx.x; e < p.sel_k; e += kThreads) sRaw[e] = lrow[e];
   __syncthreads();
   {
-    const int e = threadIdx.x;  // sel_k <= kMaxSelK = 256 = kThreads
+    const int e = threadIdx.x;  // sel_k <= kMaxSelK = 256 <= kThreads
     bool keep = false;
     if (e < p.sel_k) {
       const int v = sRaw[e];
@@ -209,35 +213,34 @@ __global__ void __launch_bounds__(kThreads)
     if (threadIdx.x == 0) {
       int tot = 0;
       for (int w = 0; w < kWarps; ++w) tot += sCnt[w];
-      sCnt[8] = tot;
+      sCnt[16] = tot;
     }
     __syncthreads();
   }
-  const int n_valid = sCnt[8];
+  const int n_valid = sCnt[16];
   const int per = (n_valid + p.n_split - 1) / p.n_split;
   const int j0 = min(part * per, n_valid), j1 = min(j0 + per, n_valid);
   const int nb = j1 - j0;
 
-  // ---- query rows in registers, in log2 units ----
-  float qr[G][DL];
+  // ---- query rows in registers (packed pairs), in log2 units ----
+  uint64_t qr[G][DL / 2];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     const __nv_bfloat16* qp = p.q + b * p.qs0 + static_cast<int64_t>(g * G + h) * p.qs1 + i * p.qs2 + lane * DL;
 #pragma unroll
     for (int e = 0; e < DL; e += 2) {
       const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qp + e));
-      qr[h][e] = f.x * p.scale_log2;
-      qr[h][e + 1] = f.y * p.scale_log2;
+      qr[h][e / 2] = f2_pack(f.x * p.scale_log2, f.y * p.scale_log2);
     }
   }
-  float acc[G][DL];
+  uint64_t acc[G][DL / 2];
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int e = 0; e < DL; ++e) acc[h][e] = 0.f;
+    for (int e = 0; e < DL / 2; ++e) acc[h][e] = 0ull;  // +0.0f in both halves
 
-  auto issue = [&](int n) {  // thread 0: K and V of the part's n-th block into stage n & 1
-    const int blk = sList[j0 + n], st = n & 1;
+  auto issue = [&](int n) {  // thread 0: K and V of the part's n-th block into stage n % kStages
+    const int blk = sList[j0 + n], st = n % C::kStages;
     mbar_arrive_expect_tx(&full[st], 2 * C::kTile);
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
@@ -247,15 +250,14 @@ __global__ void __launch_bounds__(kThreads)
   };
   int n_issued = 0;  // thread 0's count of blocks whose loads went out
   if (threadIdx.x == 0) {
-    if (nb > 0) issue(0);
-    if (nb > 1) issue(1);
-    n_issued = min(nb, 2);
+    n_issued = min(nb, C::kStages);
+    for (int n = 0; n < n_issued; ++n) issue(n);
   }
   int n_done = 0;
 
   for (int n = 0; n < nb; ++n) {
-    const int st = n & 1;
-    if (threadIdx.x == 0 && !mbar_wait(&full[st], (n >> 1) & 1, sFlag)) *sFlag = 1;
+    const int st = n % C::kStages;
+    if (threadIdx.x == 0 && !mbar_wait(&full[st], (n / C::kStages) & 1, sFlag)) *sFlag = 1;
     __syncthreads();
     if (*sFlag) break;  // uniform: every thread reads the flag after the barrier
     const uint8_t* tK = smem + C::kK + st * C::kTile;
@@ -268,15 +270,17 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll 2
     for (int kk = 0; kk < kKeysPerWarp; ++kk) {
       const int r = warp * kKeysPerWarp + kk;
-      float kx[DL];
-      load_row<DL>(tK, r, lane, kx);
+      uint64_t kx[DL / 2];
+      load_row2<DL>(tK, r, lane, kx);
       float part_dot[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float s = 0.f;
+        uint64_t s2 = f2_fma(qr[h][0], kx[0], 0ull);
 #pragma unroll
-        for (int e = 0; e < DL; ++e) s = fmaf(qr[h][e], kx[e], s);
-        part_dot[h] = s;
+        for (int e = 1; e < DL / 2; ++e) s2 = f2_fma(qr[h][e], kx[e], s2);
+        float lo, hi;
+        f2_unpack(s2, lo, hi);
+        part_dot[h] = lo + hi;
       }
       const float tot = reduce_rows<G>(part_dot, lane);
       if ((lane & (kLanesPerRow - 1)) == 0) sS[my_row * kBlk + r] = (kbase + r <= last) ? tot : -INFINITY;
@@ -296,8 +300,8 @@ __global__ void __launch_bounds__(kThreads)
       float sum = pa + pc;
 #pragma unroll
       for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
-      sS[h * kBlk + lane] = pa;
-      sS[h * kBlk + lane + 32] = pc;
+      sPT[lane * GP + h] = pa;
+      sPT[(lane + 32) * GP + h] = pc;
       __syncwarp();
       if (lane == 0) {
         const float alpha = ex2_approx(m_old - m_use);  // 0 while nothing was visible
@@ -312,26 +316,38 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float alpha = sA[h];
+      const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-      for (int e = 0; e < DL; ++e) acc[h][e] *= alpha;
+      for (int e = 0; e < DL / 2; ++e) acc[h][e] = f2_fma(acc[h][e], a2, 0ull);
     }
 #pragma unroll 2
     for (int kk = 0; kk < kKeysPerWarp; ++kk) {
       const int r = warp * kKeysPerWarp + kk;
-      float vx[DL];
-      load_row<DL>(tV, r, lane, vx);
+      uint64_t vx[DL / 2];
+      load_row2<DL>(tV, r, lane, vx);
+      float pr[GP];
+      if constexpr (GP == G && G % 4 == 0) {
+#pragma unroll
+        for (int h = 0; h < G; h += 4) {
+          const float4 f = *reinterpret_cast<const float4*>(sPT + r * GP + h);
+          pr[h] = f.x; pr[h + 1] = f.y; pr[h + 2] = f.z; pr[h + 3] = f.w;
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < G; ++h) pr[h] = sPT[r * GP + h];
+      }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float pp = sS[h * kBlk + r];
+        const uint64_t p2 = f2_pack(pr[h], pr[h]);
 #pragma unroll
-        for (int e = 0; e < DL; ++e) acc[h][e] = fmaf(pp, vx[e], acc[h][e]);
+        for (int e = 0; e < DL / 2; ++e) acc[h][e] = f2_fma(p2, vx[e], acc[h][e]);
       }
     }
     __syncthreads();  // stage st and the scores are free again
     n_done = n + 1;
-    if (threadIdx.x == 0 && n + 2 < nb) {
-      issue(n + 2);
-      n_issued = n + 3;
+    if (threadIdx.x == 0 && n + C::kStages < nb) {
+      issue(n + C::kStages);
+      n_issued = n + C::kStages + 1;
     }
   }
   const bool aborted = *sFlag != 0;
@@ -339,7 +355,7 @@ __global__ void __launch_bounds__(kThreads)
     atomicOr(p.err, MFA_DEVERR_TIMEOUT);
     // let the copies already issued land before shared memory is released
     volatile int no_abort = 0;
-    for (int n = n_done; n < n_issued; ++n) mbar_wait(&full[n & 1], (n >> 1) & 1, &no_abort);
+    for (int n = n_done; n < n_issued; ++n) mbar_wait(&full[n % C::kStages], (n / C::kStages) & 1, &no_abort);
   }
   if (aborted) return;
 
@@ -350,7 +366,12 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int e = 0; e < DL; ++e) red[(warp * 32 + lane) * kRow + h * DL + e] = acc[h][e];
+    for (int e = 0; e < DL / 2; ++e) {
+      float lo, hi;
+      f2_unpack(acc[h][e], lo, hi);
+      red[(warp * 32 + lane) * kRow + h * DL + 2 * e] = lo;
+      red[(warp * 32 + lane) * kRow + h * DL + 2 * e + 1] = hi;
+    }
   __syncthreads();
   // Element (h, dimension) = (h, DL * l + e) lives at lane l, slot h * DL + e of every warp.
   for (int it = threadIdx.x; it < G * D; it += kThreads) {
@@ -384,11 +405,11 @@ __global__ void __launch_bounds__(kThreads)
 // M = max m_s, out = sum o_s 2^(m_s - M) / sum l_s 2^(m_s - M). All parts
 // empty gives M = -FLT_MAX, weights 1 on zeros, l = 0: out = 0, lse = -inf.
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads) mfa_decode_combine(const DecParams p) {
+__global__ void __launch_bounds__(kCombineThreads) mfa_decode_combine(const DecParams p) {
   const size_t ru = blockIdx.x;  // (bg, i)
   const int bg = static_cast<int>(ru / p.Nq), i = static_cast<int>(ru % p.Nq);
   const int b = bg / p.Hkv, g = bg % p.Hkv;
-  for (int it = threadIdx.x; it < G * D; it += kThreads) {
+  for (int it = threadIdx.x; it < G * D; it += kCombineThreads) {
     const int h = it / D, d = it % D;
     float M = -FLT_MAX;
     for (int s = 0; s < p.n_split; ++s) M = fmaxf(M, p.ml_part[((ru * p.n_split + s) * G + h) * 2]);
@@ -468,10 +489,10 @@ mfa_status launch_dec(const CUtensorMap& mk, const CUtensorMap& mv, const DecPar
     attr = true;
   }
   const dim3 grid(p.n_split, p.Nq, p.B * p.Hkv);
-  mfa_decode_kernel<D, G><<<grid, kThreads, C::kBytes, s>>>(mk, mv, p);
+  mfa_decode_kernel<D, G><<<grid, kWarpsFor<D, G> * 32, C::kBytes, s>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
   if (p.n_split > 1) {
-    mfa_decode_combine<D, G><<<static_cast<unsigned>(p.B * p.Hkv * p.Nq), kThreads, 0, s>>>(p);
+    mfa_decode_combine<D, G><<<static_cast<unsigned>(p.B * p.Hkv * p.Nq), kCombineThreads, 0, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
   }
   return MFA_OK;
@@ -489,13 +510,21 @@ mfa_status launch_dec_g(const CUtensorMap& mk, const CUtensorMap& mv, const DecP
   }
 }
 
-int32_t auto_split(int64_t rows, int32_t sel_k) {
-  // enough CTAs for two per SM, at most one block per part
+// Parts per list: the fewest that give one wave of CTAs on at least 85 % of
+// the SMs (CTAs per SM from the kernel's shared memory), at most half the
+// list length. Every part pays the list deduplication, the query load and the
+// output write, so fewer and longer parts are faster once the SMs are busy
+// (decode_sel64k: 2 parts 2.35 TB/s, 4 parts 1.99, 16 parts 1.28).
+int32_t auto_split(int64_t rows, int32_t sel_k, int D) {
   const int sms = sm_count_dec() > 0 ? sm_count_dec() : 148;
-  int64_t n = (2 * sms + rows - 1) / rows;
-  if (n > sel_k) n = sel_k;
-  if (n < 1) n = 1;
-  return static_cast<int32_t>(n);
+  const int bytes = D == 128 ? DecCfg<128>::kBytes : DecCfg<256>::kBytes;
+  const int per_sm = (227 * 1024) / bytes > 0 ? (227 * 1024) / bytes : 1;
+  const int64_t target = (static_cast<int64_t>(sms) * per_sm * 85 + 99) / 100;
+  const int64_t max_ns = sel_k / 2 > 1 ? sel_k / 2 : 1;
+  int64_t ns = (target + rows - 1) / rows;
+  if (ns > max_ns) ns = max_ns;
+  if (ns < 1) ns = 1;
+  return static_cast<int32_t>(ns);
 }
 
 }  // namespace
@@ -506,7 +535,7 @@ extern "C" size_t mfa_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv,
   using namespace mfa;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || D <= 0 || sel_k <= 0 || n_split < 0 || Hq % Hkv) return 0;
   const int64_t rows = static_cast<int64_t>(B) * Hkv * Nq;
-  const int32_t ns = n_split == 0 ? auto_split(rows > 0 ? rows : 1, sel_k) : n_split;
+  const int32_t ns = n_split == 0 ? auto_split(rows > 0 ? rows : 1, sel_k, D) : n_split;
   if (ns <= 1) return 256;
   const int64_t G = Hq / Hkv;
   const size_t o = align256(static_cast<size_t>(rows * ns * G * D) * 4);
@@ -534,7 +563,7 @@ extern "C" mfa_status mfa_decode(const mfa_tensor* q, const mfa_tensor* k, const
   if (sel_k > kMaxSelK || q->B * k->H > 65535 || q->N > 65535 || k->N > (int64_t(1) << 30))
     return MFA_ERR_UNSUPPORTED;
   const int64_t rows = q->B * k->H * q->N;
-  const int32_t ns = n_split == 0 ? auto_split(rows > 0 ? rows : 1, sel_k) : n_split;
+  const int32_t ns = n_split == 0 ? auto_split(rows > 0 ? rows : 1, sel_k, static_cast<int>(q->D)) : n_split;
   if (ns > 65535) return MFA_ERR_UNSUPPORTED;
   if (ns > 1) {
     const size_t o = align256(static_cast<size_t>(rows * ns * G * q->D) * 4);

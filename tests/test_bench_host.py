@@ -57,3 +57,15 @@ def test_varlen_prefill_pairs_match_the_oracle_modes(N):
 def test_varlen_prefill_problem_is_rectangular():
     p = W.make_problem("varlen_prefill16k", N=2048, Hq=4, Hkv=2)
     assert p.q.shape[2] == p.mask.Nq and p.k.shape[2] == p.v.shape[2] == p.mask.Nk == 2048
+
+
+def test_decode_bytes_count_the_oracle_visibility():
+    import torch
+    from oracle import decode as OD
+    rng = np.random.default_rng(9)
+    sel = W.decode_selection(rng, 2, 2, 3, 1000, 8, pads=2, dups=2)
+    q = torch.zeros(2, 8, 3, 128, dtype=torch.bfloat16)
+    k = torch.zeros(2, 2, 1000, 128, dtype=torch.bfloat16)
+    keys = sum(int(OD.visible_dense(sel, b, g, 3, 1000).sum()) for b in range(2) for g in range(2))
+    expect = keys * 128 * 2 * 2 + 2 * q.numel() * 2 + 2 * 8 * 3 * 4 + sel.size * 4
+    assert bench.decode_bytes(q, k, sel) == expect
