@@ -35,14 +35,17 @@ def _f64(t) -> np.ndarray:
     return np.asarray(t, dtype=np.float64)
 
 
-def attention_rows(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, vis: np.ndarray):
+def attention_rows(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, vis: np.ndarray, bias=None):
     """Attention of some query rows of one head.
 
-    q_rows [R, d], k [Nk, d], v [Nk, dv] in float64, vis [R, Nk] bool.
+    q_rows [R, d], k [Nk, d], v [Nk, dv] in float64, vis [R, Nk] bool;
+    bias: optional [R, Nk] float64 added to the scores of visible pairs.
     Returns (out [R, dv], lse [R]).
     """
     d = q_rows.shape[1]
     s = (q_rows @ k.T) / math.sqrt(d)
+    if bias is not None:
+        s = s + bias
     s = np.where(vis, s, -np.inf)
     m = s.max(axis=1) if s.shape[1] else np.full(s.shape[0], -np.inf)
     empty = ~np.isfinite(m)
