@@ -233,6 +233,33 @@ mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v
                    const mfa_mask_desc* mask, const mfa_tensor* out, float* lse,
                    void* stream);
 
+/* Additive ALiBi bias on the scores of visible pairs, from the Ascend CANN
+ * "Mask Compression" page (ALiBi paragraphs): a per-head slope times a bias
+ * matrix, the slopes passed in. The page's figures of the bias matrices are
+ * lost; the bias of visible pair (row i, key j) is read as
+ *   MFA_BIAS_ALIBI       slope_h * (j - i)       (right-aligned)
+ *   MFA_BIAS_ALIBI_SQRT  -slope_h * sqrt(|i - j|)
+ *   MFA_BIAS_ALIBI_LEFT  slope_h * j             (left-aligned: the output of
+ *                        MFA_BIAS_ALIBI, lse larger by slope_h * i)
+ * The boolean visibility still comes from the mask description. */
+#define MFA_BIAS_NONE 0
+#define MFA_BIAS_ALIBI 1
+#define MFA_BIAS_ALIBI_SQRT 2
+#define MFA_BIAS_ALIBI_LEFT 3
+typedef struct mfa_bias {
+  int32_t kind;           /* MFA_BIAS_*                                   */
+  int32_t reserved;       /* 0                                            */
+  const float* slopes;    /* DEVICE float32 [Hq], one slope per query head */
+} mfa_bias;
+
+/* mfa_fwd with an additive bias (bias != NULL; kind MFA_BIAS_NONE is plain
+ * mfa_fwd). bf16 inputs only: fp32 inputs with a bias return
+ * MFA_ERR_UNSUPPORTED. Every computed tile, FULL or PARTIAL, adds the bias
+ * per element; the tile map is the mask's own. */
+mfa_status mfa_fwd_bias(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v,
+                        const mfa_mask_desc* mask, const mfa_bias* bias, const mfa_tensor* out, float* lse,
+                        void* stream);
+
 /* Size of the device array mfa_fwd_noalloc keeps its tile map and work
  * counters in: 16 MiB, held on every GPU where the library's kernels are
  * loaded, until the process exits. */

@@ -25,7 +25,8 @@ DEVERR_BOUNDS, DEVERR_SEL, DEVERR_TIMEOUT, DEVERR_MAP = 1, 2, 4, 8
 EXPORTS = ("mfa_abi_version", "mfa_status_string", "mfa_tile_map_bytes", "mfa_tile_map_init",
            "mfa_build_tile_map", "mfa_fwd", "mfa_fwd_noalloc", "mfa_get_device_status",
            "mfa_mask_from_sparse_mode", "mfa_bwd_workspace_bytes", "mfa_bwd", "mfa_decode_workspace_bytes",
-           "mfa_decode")
+           "mfa_decode", "mfa_fwd_bias")
+BIAS_NONE, BIAS_ALIBI, BIAS_ALIBI_SQRT, BIAS_ALIBI_LEFT = 0, 1, 2, 3
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -57,6 +58,10 @@ class MfaSparseMode(ctypes.Structure):
                 ("pre_tokens", ctypes.c_int64), ("next_tokens", ctypes.c_int64),
                 ("prefix", ctypes.c_void_p), ("seq_q", ctypes.c_void_p), ("seq_kv", ctypes.c_void_p),
                 ("n_seq", ctypes.c_int32), ("reserved2", ctypes.c_int32)]
+
+
+class MfaBias(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("reserved", ctypes.c_int32), ("slopes", ctypes.c_void_p)]
 
 
 class MfaError(RuntimeError):
@@ -104,6 +109,11 @@ def load(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.mfa_bwd.restype = ctypes.c_int
     lib.mfa_bwd.argtypes = [ctypes.POINTER(MfaTensor)] * 5 + [ctypes.c_void_p, ctypes.POINTER(MfaMaskDesc)] + \
         [ctypes.POINTER(MfaTensor)] * 3 + [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    lib.mfa_fwd_bias.restype = ctypes.c_int
+    lib.mfa_fwd_bias.argtypes = [ctypes.POINTER(MfaTensor)] * 3 + [ctypes.POINTER(MfaMaskDesc),
+                                                                   ctypes.POINTER(MfaBias),
+                                                                   ctypes.POINTER(MfaTensor), ctypes.c_void_p,
+                                                                   ctypes.c_void_p]
     lib.mfa_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.mfa_decode_workspace_bytes.argtypes = [ctypes.c_int32] * 7
     lib.mfa_decode.restype = ctypes.c_int
@@ -260,6 +270,21 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: DeviceMask, tm
                                      ctypes.byref(od), lse.data_ptr(), _stream_ptr(stream)))
 
 
+def fwd_bias(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask, tmap: TileMap, kind: int,
+             slopes: torch.Tensor, out: torch.Tensor, lse: torch.Tensor, stream=None) -> None:
+    """Forward pass with an additive ALiBi bias (kind BIAS_*, slopes: float32 device tensor [Hq])."""
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor")
+    if slopes.dtype != torch.float32 or not slopes.is_contiguous():
+        raise ValueError("slopes must be a contiguous float32 tensor")
+    dmask.desc.map = ctypes.pointer(tmap.m)
+    bias = MfaBias(kind, 0, slopes.data_ptr())
+    qd, kd, vd, od = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
+    _check("mfa_fwd_bias", load().mfa_fwd_bias(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd),
+                                               ctypes.byref(dmask.desc), ctypes.byref(bias), ctypes.byref(od),
+                                               lse.data_ptr(), _stream_ptr(stream)))
+
+
 def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: DeviceMask, block_q: int, block_k: int,
                 out: torch.Tensor, lse: torch.Tensor, dev_err: Optional[torch.Tensor] = None, stream=None) -> None:
     """Forward pass with the tile map in the library's own device array (no allocation by anyone)."""
@@ -354,12 +379,16 @@ class Attention:
     def build(self, stream=None):
         build_tile_map(self.dmask, self.tmap, stream)
 
-    def __call__(self, q, k, v, out=None, lse=None, stream=None):
+    def __call__(self, q, k, v, out=None, lse=None, stream=None, bias=None):
+        """bias: None or (kind, slopes) with kind one of BIAS_* and slopes a float32 device tensor [Hq]."""
         if out is None:
             out = torch.empty_like(q)
         if lse is None:
             lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
-        fwd(q, k, v, self.dmask, self.tmap, out, lse, stream)
+        if bias is None:
+            fwd(q, k, v, self.dmask, self.tmap, out, lse, stream)
+        else:
+            fwd_bias(q, k, v, self.dmask, self.tmap, bias[0], bias[1], out, lse, stream)
         return out, lse
 
     def backward(self, q, k, v, out, lse, dout, dq=None, dk=None, dv=None, stream=None):

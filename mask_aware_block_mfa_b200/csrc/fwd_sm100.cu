@@ -78,6 +78,8 @@ struct FwdParams {
   float* lse;
   uint32_t* err;
   uint32_t* sched;  // [0] next work item, [1] CTAs finished (map scratch words)
+  int32_t bias_kind;     // MFA_BIAS_* (kernels instantiated with kBias only)
+  const float* slopes;   // [Hq] ALiBi slopes
 };
 
 constexpr int kRing = 4;  // decoded work items in flight from the producer to the other roles
@@ -223,7 +225,8 @@ __device__ __forceinline__ uint32_t transpose32_warp(uint32_t x, int lane) {
   return x;
 }
 
-template <int D, int BK, int GP>
+// kBias: 0 none, 1 linear ALiBi (right- or left-aligned), 2 square-root ALiBi.
+template <int D, int BK, int GP, int kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     mfa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -573,6 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qi = (GP == 2) ? T.q0 + (r & 63) : T.q0 + r;
       const int head = (GP == 2) ? T.h0 + (r >> 6) : T.h0;
       const int n = T.n;
+      // ALiBi slope of this row's head in log2 units (additive bias variant only).
+      const float slope2 = kBias != 0 ? __ldg(p.slopes + head) * 1.4426950408889634f : 0.f;
       float m_run = -INFINITY, l_run = 0.f;
 
       for (int i = 0; i < n; ++i) {
@@ -670,6 +675,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int jj = 0; jj < BK; ++jj)
             if ((mrow[jj >> 5] >> (jj & 31)) & 1u) s[jj] = -INFINITY;
         }
+        // Scores in log2 units: s * scale here, or, with an additive bias,
+        // s * scale + bias(i, j) written into s (masked entries stay -inf)
+        // and a unit scale from here on.
+        float sc = p.scale_log2;
+        if constexpr (kBias == 2) {
+          const int dj0 = kt * BK - qi;  // j - i of column 0
+#pragma unroll
+          for (int jj = 0; jj < BK; ++jj)
+            s[jj] = fmaf(s[jj], sc, -slope2 * sqrtf(fabsf(static_cast<float>(dj0 + jj))));
+          sc = 1.f;
+        } else if constexpr (kBias == 1) {
+          // linear: slope (j - i); left-aligned: slope j = slope (j - i) + slope i
+          const float c0 = slope2 * static_cast<float>(p.bias_kind == MFA_BIAS_ALIBI_LEFT ? kt * BK : kt * BK - qi);
+#pragma unroll
+          for (int jj = 0; jj < BK; ++jj) s[jj] = fmaf(s[jj], sc, fmaf(slope2, static_cast<float>(jj), c0));
+          sc = 1.f;
+        }
         // Row max with 3-input max instructions over four independent chains.
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -677,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int a = 0; a < 4; ++a) mx4[a] = fmax3(mx4[a], s[jj + 2 * a], s[jj + 2 * a + 1]);
         const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]);
-        const float mx_s = mx * p.scale_log2;
+        const float mx_s = mx * sc;
         const bool need = mx_s > m_run + kRescaleThreshold;
         const float m_new = need ? mx_s : m_run;
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
@@ -692,8 +714,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
-            const float e0 = ex2_approx(fmaf(s[c * 32 + 2 * u], p.scale_log2, -m_use));
-            const float e1 = ex2_approx(fmaf(s[c * 32 + 2 * u + 1], p.scale_log2, -m_use));
+            const float e0 = ex2_approx(fmaf(s[c * 32 + 2 * u], sc, -m_use));
+            const float e1 = ex2_approx(fmaf(s[c * 32 + 2 * u + 1], sc, -m_use));
             sum4[u & 3] += e0 + e1;
             pk[u] = pack_bf16x2(e0, e1);
           }
@@ -865,31 +887,62 @@ int sm_count() {
   return n;
 }
 
-template <int D, int BK, int GP>
-mfa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
-                  cudaStream_t s) {
+template <int D, int BK, int GP, int kBias>
+mfa_status launch_b(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
+                    cudaStream_t s) {
   using C = Cfg<D, BK>;
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(mfa_fwd_kernel<D, BK, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(mfa_fwd_kernel<D, BK, GP, kBias>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kAlloc) != cudaSuccess)
       return MFA_ERR_CUDA;
     attr_set = true;
   }
   const int sms = sm_count();
   if (sms <= 0) return MFA_ERR_CUDA;
   const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: at most one CTA per SM
-  mfa_fwd_kernel<D, BK, GP><<<grid, kThreads, C::kAlloc, s>>>(mq, mk, mv, p);
+  mfa_fwd_kernel<D, BK, GP, kBias><<<grid, kThreads, C::kAlloc, s>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
+}
+
+template <int D, int BK, int GP>
+mfa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
+                  cudaStream_t s) {
+  if (p.bias_kind == MFA_BIAS_NONE) return launch_b<D, BK, GP, 0>(mq, mk, mv, p, s);
+  if (p.bias_kind == MFA_BIAS_ALIBI_SQRT) return launch_b<D, BK, GP, 2>(mq, mk, mv, p, s);
+  return launch_b<D, BK, GP, 1>(mq, mk, mv, p, s);
 }
 
 }  // namespace
 }  // namespace mfa
 
+namespace mfa {
+namespace {
+mfa_status fwd_impl(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v, const mfa_mask_desc* mask,
+                    const mfa_bias* bias, const mfa_tensor* out, float* lse, void* stream);
+}  // namespace
+}  // namespace mfa
+
 extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v,
                               const mfa_mask_desc* mask, const mfa_tensor* out, float* lse, void* stream) {
-  using namespace mfa;
+  return mfa::fwd_impl(q, k, v, mask, nullptr, out, lse, stream);
+}
+
+extern "C" mfa_status mfa_fwd_bias(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v,
+                                   const mfa_mask_desc* mask, const mfa_bias* bias, const mfa_tensor* out, float* lse,
+                                   void* stream) {
+  if (!bias) return MFA_ERR_INVALID_ARG;
+  return mfa::fwd_impl(q, k, v, mask, bias, out, lse, stream);
+}
+
+namespace mfa {
+namespace {
+mfa_status fwd_impl(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v, const mfa_mask_desc* mask,
+                    const mfa_bias* bias, const mfa_tensor* out, float* lse, void* stream) {
   mfa_status st;
+  const int32_t bias_kind = bias ? bias->kind : MFA_BIAS_NONE;
+  if (bias_kind < MFA_BIAS_NONE || bias_kind > MFA_BIAS_ALIBI_LEFT) return MFA_ERR_INVALID_ARG;
+  if (bias_kind != MFA_BIAS_NONE && !bias->slopes) return MFA_ERR_INVALID_ARG;
   if ((st = check_tensor(q)) != MFA_OK || (st = check_tensor(k)) != MFA_OK || (st = check_tensor(v)) != MFA_OK ||
       (st = check_tensor(out)) != MFA_OK)
     return st;
@@ -908,7 +961,10 @@ extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   if (mask->Hm != 1 && mask->Hm != q->H) return MFA_ERR_SHAPE_MISMATCH;
   if (q->D != 64 && q->D != 128) return MFA_ERR_UNSUPPORTED;
   if (q->N > (int64_t(1) << 30) || k->N > (int64_t(1) << 30) || q->H > 65535) return MFA_ERR_UNSUPPORTED;
-  if (q->dtype == MFA_F32) return launch_fwd_f32(q, k, v, mask, map, out, lse, static_cast<cudaStream_t>(stream));
+  if (q->dtype == MFA_F32) {
+    if (bias_kind != MFA_BIAS_NONE) return MFA_ERR_UNSUPPORTED;  // the fp32 path takes no bias
+    return launch_fwd_f32(q, k, v, mask, map, out, lse, static_cast<cudaStream_t>(stream));
+  }
   const int G = static_cast<int>(q->H / k->H);
   const int GP = map->block_q == 64 ? 2 : 1;
   if (GP == 2 && (mask->Hm != 1 || G % 2 != 0)) return MFA_ERR_UNSUPPORTED;
@@ -948,6 +1004,8 @@ extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   p.lse = lse;
   p.err = map->err;
   p.sched = map->err + 1;
+  p.bias_kind = bias_kind;
+  p.slopes = bias_kind != MFA_BIAS_NONE ? bias->slopes : nullptr;
   if (n_items64 <= 0) return MFA_OK;
   if (n_items64 > 0x7fffffff) return MFA_ERR_UNSUPPORTED;
   p.n_items = static_cast<int32_t>(n_items64);
@@ -965,3 +1023,6 @@ extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mf
   if (D == 64 && BK == 128) return GP == 2 ? launch<64, 128, 2>(mq, mk, mv, p, s) : launch<64, 128, 1>(mq, mk, mv, p, s);
   return GP == 2 ? launch<64, 64, 2>(mq, mk, mv, p, s) : launch<64, 64, 1>(mq, mk, mv, p, s);
 }
+
+}  // namespace
+}  // namespace mfa

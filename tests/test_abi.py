@@ -47,8 +47,10 @@ def test_struct_layouts_match_header(tmp_path):
 #include "mfa.h"
 #define F(T, f) printf(#T "." #f " %zu\n", offsetof(T, f))
 int main(void) {
-  printf("mfa_tensor %zu\nmfa_tile_map %zu\nmfa_mask_desc %zu\nmfa_sparse_mode %zu\n",
-         sizeof(mfa_tensor), sizeof(mfa_tile_map), sizeof(mfa_mask_desc), sizeof(mfa_sparse_mode));
+  printf("mfa_tensor %zu\nmfa_tile_map %zu\nmfa_mask_desc %zu\nmfa_sparse_mode %zu\nmfa_bias %zu\n",
+         sizeof(mfa_tensor), sizeof(mfa_tile_map), sizeof(mfa_mask_desc), sizeof(mfa_sparse_mode),
+         sizeof(mfa_bias));
+  F(mfa_bias, kind); F(mfa_bias, slopes);
   F(mfa_sparse_mode, pre_tokens); F(mfa_sparse_mode, prefix); F(mfa_sparse_mode, seq_kv); F(mfa_sparse_mode, n_seq);
   F(mfa_tensor, data); F(mfa_tensor, B); F(mfa_tensor, stride);
   F(mfa_tile_map, kind); F(mfa_tile_map, kminmax); F(mfa_tile_map, err);
@@ -62,11 +64,12 @@ int main(void) {
     assert int(got["mfa_tile_map"]) == ctypes.sizeof(B.MfaTileMap)
     assert int(got["mfa_mask_desc"]) == ctypes.sizeof(B.MfaMaskDesc)
     assert int(got["mfa_sparse_mode"]) == ctypes.sizeof(B.MfaSparseMode)
+    assert int(got["mfa_bias"]) == ctypes.sizeof(B.MfaBias)
     for key, val in got.items():
         if "." in key:
             struct, field = key.split(".")
             cls = {"mfa_tensor": B.MfaTensor, "mfa_tile_map": B.MfaTileMap, "mfa_mask_desc": B.MfaMaskDesc,
-                   "mfa_sparse_mode": B.MfaSparseMode}[struct]
+                   "mfa_sparse_mode": B.MfaSparseMode, "mfa_bias": B.MfaBias}[struct]
             assert getattr(cls, field).offset == int(val), key
 
 
@@ -269,3 +272,22 @@ def test_decode_rejects_bad_arguments_on_host(lib):
     assert call(k=k0, v=v0) == B.MFA_ERR_UNSUPPORTED                             # no keys
     f32 = _fake_tensor(1, 8, 1, 256, dtype=B.MFA_F32)
     assert call(q=f32) == B.MFA_ERR_UNSUPPORTED
+
+
+def test_fwd_bias_rejects_bad_arguments_on_host(lib):
+    m = _fake_map(lib)
+    q, k, v, o = _fake_tensor(1, 8, 512, 128), _fake_tensor(1, 2, 512, 128), _fake_tensor(1, 2, 512, 128), \
+        _fake_tensor(1, 8, 512, 128)
+    d = _fake_mask(m)
+
+    def call(bias, q=q, k=k, v=v, o=o):
+        return lib.mfa_fwd_bias(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.byref(d),
+                                None if bias is None else ctypes.byref(bias), ctypes.byref(o), 0x7200_0000_0000, None)
+
+    assert call(None) == B.MFA_ERR_INVALID_ARG
+    assert call(B.MfaBias(7, 0, 0x7600_0000_0000)) == B.MFA_ERR_INVALID_ARG       # unknown kind
+    assert call(B.MfaBias(B.BIAS_ALIBI, 0, None)) == B.MFA_ERR_INVALID_ARG        # no slopes
+    f32 = [_fake_tensor(1, h, 512, 128, dtype=B.MFA_F32) for h in (8, 2, 2, 8)]
+    mf = _fake_map(lib, bq=128)
+    d = _fake_mask(mf)
+    assert call(B.MfaBias(B.BIAS_ALIBI, 0, 0x7600_0000_0000), *f32) == B.MFA_ERR_UNSUPPORTED  # fp32 + bias
