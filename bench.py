@@ -582,6 +582,8 @@ def main():
     ap.add_argument("--reference-heads", type=int, default=1, help="query heads per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--bias", default="none", choices=["none", "alibi", "alibi_sqrt", "alibi_left"],
+                    help="additive ALiBi bias in the forward pass (slopes 2^(-8h/Hq))")
     ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "decode"],
                     help="fwd: tile map + forward (the headline); bwd: the gradient pass alone; "
                          "decode: selected-key decode (decode workloads)")
@@ -632,6 +634,11 @@ def main():
         return B.DeviceMask(prob.mask, dev)
 
     att = B.Attention(device_mask(), bq, bk, device=dev)
+    bias = None
+    if args.bias != "none":
+        kind = {"alibi": B.BIAS_ALIBI, "alibi_sqrt": B.BIAS_ALIBI_SQRT, "alibi_left": B.BIAS_ALIBI_LEFT}[args.bias]
+        slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / Hq) for h in range(Hq)], dtype=torch.float32, device=dev)
+        bias = (kind, slopes)
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -641,7 +648,7 @@ def main():
         if sparse:
             att.dmask.convert()
         att.build()
-        att(q, k, v, out, lse)
+        att(q, k, v, out, lse, bias=bias)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -659,7 +666,7 @@ def main():
         with torch.cuda.graph(g_step, stream=cap):
             step()
         with torch.cuda.graph(g_fwd, stream=cap):
-            att(q, k, v, out, lse)
+            att(q, k, v, out, lse, bias=bias)
     stream.wait_stream(cap)
     for _ in range(args.warmup):
         g_step.replay()
@@ -720,7 +727,7 @@ def main():
         k.copy_(hk, non_blocking=True)
         v.copy_(hv, non_blocking=True)
         att_e.build(stream)
-        att_e(q, k, v, out, lse, stream)
+        att_e(q, k, v, out, lse, stream, bias=bias)
         ho.copy_(out, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
         z.record(stream)
@@ -739,7 +746,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, "desc": W.WORKLOADS[args.workload], "B": Bsz, "Hq": Hq, "Hkv": Hkv,
-                   "N": N, "Nk": prob.Nk, "d": d, "block_q": bq, "block_k": bk, "seed": prob.seed, "visible_pairs": pairs,
+                   "N": N, "Nk": prob.Nk, "d": d, "block_q": bq, "block_k": bk, "bias": args.bias, "seed": prob.seed, "visible_pairs": pairs,
                    "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}",
                    "launch": "each step replayed as a CUDA graph (" + ("sparse-mode conversion + " if sparse else "")
                              + "map build + forward)"},
