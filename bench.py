@@ -51,8 +51,8 @@ METRIC = "effective TFLOP/s (visible pairs only) and % of B200 bf16 tensor peak"
 # on; a changed kernel reports traffic as null until it is captured again.
 KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/fwd_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh")
 NCU_TRAFFIC = {
-    "doc8k": (135_656_192, "80823225e4d4639b"),
-    "doc32k": (1_023_853_056, "80823225e4d4639b"),
+    "doc8k": (135_804_672, "ee84eb1bb5741042"),
+    "doc32k": (1_031_209_472, "ee84eb1bb5741042"),
 }
 # The same for the gradient kernel (mfa_bwd_kernel) of the backward pass.
 BWD_KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/bwd_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh",
@@ -60,6 +60,13 @@ BWD_KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/bwd_sm100.cu", "mask_aware
 BWD_NCU_TRAFFIC = {
     "doc8k": (842_567_936, "e45bc9d337ef5356"),
     "doc32k": (2_108_606_464, "e45bc9d337ef5356"),
+}
+
+
+# The same for the decode kernel (mfa_decode_kernel) of --pass decode.
+DEC_KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/decode_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh")
+DEC_NCU_TRAFFIC = {
+    "decode_sel64k": (138_088_960, "9b364fe4d18fa820"),
 }
 
 
@@ -553,7 +560,9 @@ def run_decode(args, rank, world, local):
                    "algorithmic_bytes": nbytes, "l2": "flushed between timed steps (256 MiB write)",
                    "parallelism": f"replicas x{world}", "launch": "each step replayed as a CUDA graph"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "peak_kind": f"{src} HBM copy bandwidth"},
+                     "traffic": ncu_traffic(args.workload, DEC_NCU_TRAFFIC, DEC_KERNEL_SOURCES),
+                     "peak_kind": f"{src} HBM copy bandwidth; achieved over the decode call (decode + combine), "
+                                  "traffic of the decode kernel"},
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": hq.nbytes + hsel.nbytes,
                 "d2h_bytes_per_step": ho.nbytes + hl.nbytes, "ms": statistics.mean(e2e_ms),
                 "note": "cache resident in HBM; queries and lists copied in, out and lse copied back"},

@@ -31,6 +31,11 @@ def test_ncu_traffic_follows_the_kernel_digest():
     for name, (nbytes, dig) in bench.NCU_TRAFFIC.items():
         assert nbytes > 0 and len(dig) == 16
         assert bench.ncu_traffic(name) == (nbytes if dig == digest else None)
+    dec_digest = bench.kernel_digest(bench.DEC_KERNEL_SOURCES)
+    for name, (nbytes, dig) in bench.DEC_NCU_TRAFFIC.items():
+        assert nbytes > 0 and len(dig) == 16
+        assert bench.ncu_traffic(name, bench.DEC_NCU_TRAFFIC, bench.DEC_KERNEL_SOURCES) == \
+            (nbytes if dig == dec_digest else None)
     bwd_digest = bench.kernel_digest(bench.BWD_KERNEL_SOURCES)
     assert bwd_digest != digest
     for name, (nbytes, dig) in bench.BWD_NCU_TRAFFIC.items():
