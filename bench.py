@@ -70,6 +70,23 @@ DEC_NCU_TRAFFIC = {
 }
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest x over the ranks of the default process group (x itself
+    without one): the job's time is its slowest rank's."""
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: float, world: int, steps: int, max_total_ms: float) -> float:
+    """Units per second of the whole job: every rank processes the same units
+    per step (replicas, weak scaling), timed by the slowest rank."""
+    return units_per_rank_step * world * steps / (max_total_ms * 1e-3)
+
+
 def kernel_digest(sources=KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
     root = os.path.dirname(os.path.abspath(__file__))
@@ -337,12 +354,9 @@ def run_backward(args, prob, pairs, rank, world, local):
         raise RuntimeError("device error word set during the timed steps")
     ms = [e0.elapsed_time(e1) for e0, e1 in evs]
     total_ms = sum(ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
-    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    value = whole_job_rate(flops, world, args.steps, total_ms) / 1e12
     achieved = flops / (statistics.mean(ms) * 1e-3) / 1e12
     burst, sustained, src = peaks()
 
@@ -518,11 +532,8 @@ def run_decode(args, rank, world, local):
         raise RuntimeError("device error bits set during the timed steps")
     ms = [e0.elapsed_time(e1) for e0, e1 in evs]
     total_ms = sum(ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = nbytes * world * args.steps / (total_ms * 1e-3) / 1e9
+    total_ms = max_over_ranks(total_ms, dev)
+    value = whole_job_rate(nbytes, world, args.steps, total_ms) / 1e9
     achieved = nbytes / (statistics.mean(ms) * 1e-3) / 1e9
     peak, src = hbm_peak()
     # End to end: the cache stays resident (as in serving); each step copies the
@@ -707,12 +718,9 @@ def main():
     step_ms = [e0.elapsed_time(e1) for (e0, e1) in ev_step]
     fwd_ms = [e0.elapsed_time(e1) for (e0, e1) in ev_fwd]
     total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
-    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    value = whole_job_rate(flops, world, args.steps, total_ms) / 1e12
     fwd_avg_ms = sum(fwd_ms) / len(fwd_ms)
     achieved = flops / (fwd_avg_ms * 1e-3) / 1e12
     burst, sustained, src = peaks()
