@@ -55,3 +55,24 @@ def test_zero_slopes_match_the_plain_forward():
     o1, l1 = att(q, k, v, bias=(B.BIAS_ALIBI, torch.zeros(4, dtype=torch.float32, device="cuda")))
     assert float((o0.float() - o1.float()).abs().max()) <= 1e-2
     assert float((l0 - l1).abs().max()) <= 1e-5
+
+
+@pytest.mark.parametrize("kind", KINDS[:2], ids=["linear", "sqrt"])
+def test_bias_full_size_sampled(kind):
+    """doc32k (the bench's 64 x 128 tiles, 32 heads) with the bench's slopes
+    2^(-8h/32): sampled rows of a few heads against the oracle."""
+    import bench
+    from .gpu_util import sample_rows
+    prob = W.make_problem("doc32k")
+    Bsz, Hq, Hkv, N, d = prob.shape
+    bq, bk = bench.BLOCKS["doc32k"]
+    slopes = OBias.alibi_slopes(Hq)
+    att = B.Attention(prob.mask, bq, bk)
+    att.build()
+    out, lse = att(prob.q.cuda(), prob.k.cuda(), prob.v.cuda(),
+                   bias=(kind[0], torch.tensor(slopes, dtype=torch.float32, device="cuda")))
+    assert B.device_status(att.tmap) == 0
+    rows = sample_rows(N, 48, np.random.default_rng(24))
+    heads = [0, 7, 31]
+    ref_out, ref_lse = OBias.attention_bias(prob.q, prob.k, prob.v, prob.mask, kind[1], slopes, rows=rows, heads=heads)
+    compare_attention(out.float().cpu()[:, heads][:, :, rows], lse.cpu()[:, heads][:, :, rows], ref_out, ref_lse)

@@ -75,3 +75,25 @@ def test_attention_matches_the_oracle(case):
         compare_map({key: val.cpu().numpy() for key, val in att.tmap.arrays().items()}, as_desc, bq, bk)
         ref_out, ref_lse = oracle_rows(prob, None)
         compare_attention(out.float().cpu(), lse.cpu(), ref_out, ref_lse)
+
+
+def test_varlen_prefill_full_size_sampled():
+    """The bench's varlen_prefill16k workload (sparseMode 7, Nq 8000 x Nk 16384,
+    32 query heads over 8 key/value heads) at the bench's 64 x 128 tiles:
+    sampled rows of a few heads against the oracle's mode expansion."""
+    import bench
+    prob = W.make_problem("varlen_prefill16k")
+    m = prob.mask
+    bq, bk = bench.BLOCKS["varlen_prefill16k"]
+    dev = B.SparseModeMask(**m.fields())
+    att = B.Attention(dev, bq, bk)
+    att.build()
+    out, lse = att(prob.q.cuda(), prob.k.cuda(), prob.v.cuda())
+    assert B.device_status(att.tmap) == 0
+    rng = np.random.default_rng(23)
+    rows = np.unique(np.concatenate([[0, 63, 64, m.Nq - 1], rng.choice(m.Nq, 60, replace=False)]))
+    heads = [0, 13, 31]
+    ref = SM.SparseMode(**m.fields())
+    prob_o = W.Problem("varlen_prefill16k", prob.q, prob.k, prob.v, ref, prob.seed)
+    ref_out, ref_lse = oracle_rows(prob_o, rows, heads)
+    compare_attention(out.float().cpu()[:, heads][:, :, rows], lse.cpu()[:, heads][:, :, rows], ref_out, ref_lse)
