@@ -22,13 +22,17 @@
 //      position dropped) and the part's share of it taken.
 //   2. K and V blocks arrive by TMA (64-column SW128 boxes) in a two-stage ring.
 //   3. Scores: lane l holds head dimensions [DL l, DL l + DL) of all G query
-//      rows in registers (DL = D / 32); warp w takes keys 8w .. 8w + 7 of the
+//      rows in registers (DL = D / 32); each warp takes 64 / warps keys of the
 //      block, reads each key row once (conflict-free through the swizzle) and
 //      reduces the G partial dot products across lanes by halving transposes
 //      (G - 1 + 5 - log2 G shuffles).
-//   4. Online softmax per query row (one warp per row), in log2 units.
-//   5. P.V: lane l owns the same head dimensions of all G rows; warp w adds
-//      its 8 keys; the 8 warps' partial outputs are summed once at the end.
+//   4. Online softmax per warp: each warp keeps its own running max and sum
+//      of every query row and its own partial outputs over the keys it
+//      handles (a split-K inside the CTA), so no block-wide barrier runs per
+//      block; a stage is released by one arrival per warp.
+//   5. P.V: lane l owns the same head dimensions of all G rows for the
+//      warp's keys; the warps' partials are combined once at the end, each
+//      rescaled by 2^(its max - the row's max).
 #include <cfloat>
 #include <climits>
 #include <cmath>
@@ -73,15 +77,16 @@ struct DecCfg {
   static constexpr int kStages = 3;                  // K/V ring: two blocks in flight while one is used
   static constexpr int kK = 0;                       // [kStages]
   static constexpr int kV = kK + kStages * kTile;    // [kStages]
-  static constexpr int kS = kV + kStages * kTile;    // scores [16][64] fp32, then P [64][16]
+  static constexpr int kS = kV + kStages * kTile;    // list scratch, then per-warp (m, l) at the end
   static constexpr int kList = kS + 2 * 16 * kBlk * 4;  // deduplicated list [kMaxSelK]
   static constexpr int kMisc = kList + kMaxSelK * 4; // softmax state, counters, barriers
   static constexpr int kBytes = kMisc + 1024;
-  // The final cross-warp sum of the outputs reuses the K/V ring and the score
-  // and list space after it, none of which the epilogue reads: 16 warps with
-  // G * D <= 1024 or 8 warps with G * D <= 2048.
-  static_assert(16 * 32 * (1024 / D * kDL + 1) * 4 <= kMisc, "output reduction space (16 warps)");
-  static_assert(8 * 32 * (2048 / D * kDL + 1) * 4 <= kMisc, "output reduction space (8 warps)");
+  // The final combine of the warps' outputs reuses the K/V ring (16 warps with
+  // G * D <= 1024 or 8 warps with G * D <= 2048); the warps' (m, l) go to the
+  // space after the ring.
+  static_assert(16 * 32 * (1024 / D * kDL + 1) * 4 <= kS, "output reduction space (16 warps)");
+  static_assert(8 * 32 * (2048 / D * kDL + 1) * 4 <= kS, "output reduction space (8 warps)");
+  static_assert(2 * 16 * 16 * 4 <= kList - kS, "per-warp (m, l)");
 };
 
 // Element offset of head dimensions [c0, c0 + n) of key row r in a K/V block
@@ -149,6 +154,17 @@ __device__ __forceinline__ int row_of_lane(int lane) {
   return idx;
 }
 
+// The first lane that holds row h's total after reduce_rows: h's bits from the
+// most significant down sit at lane bits 4, 3, ... (the inverse of row_of_lane).
+template <int G>
+__device__ __forceinline__ int owner_lane(int h) {
+  constexpr int lg = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
+  int lane = 0;
+#pragma unroll
+  for (int s = 0; s < lg; ++s) lane |= ((h >> (lg - 1 - s)) & 1) << (4 - s);
+  return lane;
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(kWarpsFor<D, G> * 32, 1)
     mfa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -158,35 +174,30 @@ __global__ void __launch_bounds__(kWarpsFor<D, G> * 32, 1)
   constexpr int kWarps = kWarpsFor<D, G>;
   constexpr int kThreads = kWarps * 32;
   constexpr int kKeysPerWarp = kBlk / kWarps;
-  constexpr int GP = (G + 3) / 4 * 4;  // P row stride (float4 loads)
+  constexpr int kCk = kKeysPerWarp < 4 ? kKeysPerWarp : 4;  // keys per softmax step
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = blockIdx.x, i = blockIdx.y;
   const int bg = blockIdx.z, b = bg / p.Hkv, g = bg % p.Hkv;
   const size_t row_unit = (static_cast<size_t>(bg) * p.Nq + i);
 
-  float* sS = reinterpret_cast<float*>(smem + C::kS);          // [G][64] scores
-  float* sPT = sS + 16 * kBlk;                                 // [64][GP] P, key-major
   int* sList = reinterpret_cast<int*>(smem + C::kList);
-  float* sM = reinterpret_cast<float*>(smem + C::kMisc);       // [16] running max (log2 units)
-  float* sL = sM + 16;                                         // [16] running sum
-  float* sA = sL + 16;                                         // [16] rescale factor of this block
-  int* sCnt = reinterpret_cast<int*>(sA + 16);                 // [kWarps] list compaction, [16] total
+  int* sCnt = reinterpret_cast<int*>(smem + C::kMisc + 192);   // [kWarps] list compaction, [16] total
   volatile int* sFlag = reinterpret_cast<volatile int*>(sCnt + 20);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kMisc + 512);  // [kStages]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kMisc + 512);  // [kStages] block landed
+  uint64_t* empty = full + C::kStages;                                   // [kStages] every warp done with it
 
   if ((smem_u32(smem) & 1023u) != 0u) {  // SW128 boxes need a 1024-aligned base (uniform check)
     if (threadIdx.x == 0) atomicOr(p.err, MFA_DEVERR_TIMEOUT);
     return;
   }
   if (threadIdx.x == 0) {
-    for (int st = 0; st < C::kStages; ++st) mbar_init(&full[st], 1);
+    for (int st = 0; st < C::kStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kWarps);
+    }
     *sFlag = 0;
     fence_mbarrier_init();
-  }
-  if (threadIdx.x < 16) {
-    sM[threadIdx.x] = -INFINITY;
-    sL[threadIdx.x] = 0.f;
   }
 
   // ---- 1. the row's deduplicated list ----
@@ -253,23 +264,37 @@ __global__ void __launch_bounds__(kWarpsFor<D, G> * 32, 1)
     n_issued = min(nb, C::kStages);
     for (int n = 0; n < n_issued; ++n) issue(n);
   }
-  int n_done = 0;
+  int n_done = 0;  // blocks this warp has finished
 
+  // Per-warp online softmax: every warp keeps its own running max and sum of
+  // each query row (in every lane) and its own partial outputs, over the keys
+  // it handles; the warps are combined once after the last block. No
+  // block-wide barrier is needed per block: a stage is released by one
+  // arrival per warp, and thread 0 refills it when all have arrived.
+  float m_w[G], l_w[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m_w[h] = -INFINITY;
+    l_w[h] = 0.f;
+  }
   for (int n = 0; n < nb; ++n) {
     const int st = n % C::kStages;
-    if (threadIdx.x == 0 && !mbar_wait(&full[st], (n / C::kStages) & 1, sFlag)) *sFlag = 1;
-    __syncthreads();
-    if (*sFlag) break;  // uniform: every thread reads the flag after the barrier
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (n / C::kStages) & 1, sFlag))) {
+      *sFlag = 1;
+      break;
+    }
     const uint8_t* tK = smem + C::kK + st * C::kTile;
     const uint8_t* tV = smem + C::kV + st * C::kTile;
     const int kbase = sList[j0 + n] * kBlk;
 
-    // ---- 3. scores of this warp's 8 keys ----
-    const int my_row = row_of_lane<G>(lane);
-    constexpr int kLanesPerRow = 32 / G;
-#pragma unroll 2
-    for (int kk = 0; kk < kKeysPerWarp; ++kk) {
-      const int r = warp * kKeysPerWarp + kk;
+    // The warp's keys in chunks of kCk: scores, softmax update, P.V.
+#pragma unroll
+    for (int kc = 0; kc < kKeysPerWarp; kc += kCk) {
+    // ---- 3. scores of this chunk, gathered into every lane ----
+    float tot[kCk];
+#pragma unroll
+    for (int kk = 0; kk < kCk; ++kk) {
+      const int r = warp * kKeysPerWarp + kc + kk;
       uint64_t kx[DL / 2];
       load_row2<DL>(tK, r, lane, kx);
       float part_dot[G];
@@ -282,74 +307,65 @@ __global__ void __launch_bounds__(kWarpsFor<D, G> * 32, 1)
         f2_unpack(s2, lo, hi);
         part_dot[h] = lo + hi;
       }
-      const float tot = reduce_rows<G>(part_dot, lane);
-      if ((lane & (kLanesPerRow - 1)) == 0) sS[my_row * kBlk + r] = (kbase + r <= last) ? tot : -INFINITY;
+      tot[kk] = reduce_rows<G>(part_dot, lane);
     }
-    __syncthreads();
-
-    // ---- 4. online softmax, one warp per query row ----
-    for (int h = warp; h < G; h += kWarps) {
-      const float a = sS[h * kBlk + lane], c = sS[h * kBlk + lane + 32];
-      float mx = fmaxf(a, c);
-#pragma unroll
-      for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
-      const float m_old = sM[h];
-      const float m_new = fmaxf(m_old, mx);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float pa = ex2_approx(a - m_use), pc = ex2_approx(c - m_use);
-      float sum = pa + pc;
-#pragma unroll
-      for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, d);
-      sPT[lane * GP + h] = pa;
-      sPT[(lane + 32) * GP + h] = pc;
-      __syncwarp();
-      if (lane == 0) {
-        const float alpha = ex2_approx(m_old - m_use);  // 0 while nothing was visible
-        sA[h] = alpha;
-        sL[h] = sL[h] * alpha + sum;
-        sM[h] = m_new;
-      }
-    }
-    __syncthreads();
-
-    // ---- 5. P.V of this warp's 8 keys ----
+    float pk[G][kCk];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const float alpha = sA[h];
-      const uint64_t a2 = f2_pack(alpha, alpha);
+      // ---- 4. online softmax of row h over these keys ----
+      float mx = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < DL / 2; ++e) acc[h][e] = f2_fma(acc[h][e], a2, 0ull);
+      for (int kk = 0; kk < kCk; ++kk) {
+        const float v = __shfl_sync(0xffffffffu, tot[kk], owner_lane<G>(h));
+        pk[h][kk] = (kbase + warp * kKeysPerWarp + kc + kk <= last) ? v : -INFINITY;
+        mx = fmaxf(mx, pk[h][kk]);
+      }
+      const float m_new = fmaxf(m_w[h], mx);
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = ex2_approx(m_w[h] - m_use);  // 0 while nothing was visible
+      float sum = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < kCk; ++kk) {
+        pk[h][kk] = ex2_approx(pk[h][kk] - m_use);
+        sum += pk[h][kk];
+      }
+      l_w[h] = l_w[h] * alpha + sum;
+      m_w[h] = m_new;
+      if (alpha != 1.f) {  // the same in every lane: no divergence
+        const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+        for (int e = 0; e < DL / 2; ++e) acc[h][e] = f2_fma(acc[h][e], a2, 0ull);
+      }
     }
-#pragma unroll 2
-    for (int kk = 0; kk < kKeysPerWarp; ++kk) {
-      const int r = warp * kKeysPerWarp + kk;
+
+    // ---- 5. P.V of these keys ----
+#pragma unroll
+    for (int kk = 0; kk < kCk; ++kk) {
+      const int r = warp * kKeysPerWarp + kc + kk;
       uint64_t vx[DL / 2];
       load_row2<DL>(tV, r, lane, vx);
-      float pr[GP];
-      if constexpr (GP == G && G % 4 == 0) {
-#pragma unroll
-        for (int h = 0; h < G; h += 4) {
-          const float4 f = *reinterpret_cast<const float4*>(sPT + r * GP + h);
-          pr[h] = f.x; pr[h + 1] = f.y; pr[h + 2] = f.z; pr[h + 3] = f.w;
-        }
-      } else {
-#pragma unroll
-        for (int h = 0; h < G; ++h) pr[h] = sPT[r * GP + h];
-      }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const uint64_t p2 = f2_pack(pr[h], pr[h]);
+        const uint64_t p2 = f2_pack(pk[h][kk], pk[h][kk]);
 #pragma unroll
         for (int e = 0; e < DL / 2; ++e) acc[h][e] = f2_fma(p2, vx[e], acc[h][e]);
       }
     }
-    __syncthreads();  // stage st and the scores are free again
+    }  // key chunks
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
     n_done = n + 1;
+    // Thread 0 refills stage st with block n + kStages once every warp has released it.
     if (threadIdx.x == 0 && n + C::kStages < nb) {
-      issue(n + C::kStages);
-      n_issued = n + C::kStages + 1;
+      if (mbar_wait(&empty[st], (n / C::kStages) & 1, sFlag)) {
+        issue(n + C::kStages);
+        n_issued = n + C::kStages + 1;
+      } else {
+        *sFlag = 1;
+      }
     }
   }
+  __syncthreads();
   const bool aborted = *sFlag != 0;
   if (aborted && threadIdx.x == 0) {
     atomicOr(p.err, MFA_DEVERR_TIMEOUT);
@@ -359,10 +375,12 @@ __global__ void __launch_bounds__(kWarpsFor<D, G> * 32, 1)
   }
   if (aborted) return;
 
-  // ---- cross-warp sum of the outputs (reusing the K/V ring and the score space) ----
+  // ---- combine the warps (reusing the K/V ring and the score space) ----
   // Rows of G * DL + 1 floats, so the 32 lanes' stores fall in different banks.
   constexpr int kRow = G * DL + 1;
-  float* red = reinterpret_cast<float*>(smem + C::kK);  // [kWarps][32 lanes][kRow]
+  float* red = reinterpret_cast<float*>(smem + C::kK);   // [kWarps][32 lanes][kRow]
+  float* sMw = reinterpret_cast<float*>(smem + C::kS);    // [kWarps][G] running max
+  float* sLw = sMw + kWarps * G;                          // [kWarps][G] running sum
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
@@ -372,15 +390,29 @@ __global__ void __launch_bounds__(kWarpsFor<D, G> * 32, 1)
       red[(warp * 32 + lane) * kRow + h * DL + 2 * e] = lo;
       red[(warp * 32 + lane) * kRow + h * DL + 2 * e + 1] = hi;
     }
+  if (lane == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      sMw[warp * G + h] = m_w[h];
+      sLw[warp * G + h] = l_w[h];
+    }
+  }
   __syncthreads();
   // Element (h, dimension) = (h, DL * l + e) lives at lane l, slot h * DL + e of every warp.
   for (int it = threadIdx.x; it < G * D; it += kThreads) {
     const int h = it / D, d = it % D;
     const int l = d / DL, e = d % DL;
-    float o = 0.f;
+    float m = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) o += red[(w * 32 + l) * kRow + h * DL + e];
-    const float m = sM[h], lsum = sL[h];
+    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, sMw[w * G + h]);
+    const float m_use = m == -INFINITY ? 0.f : m;
+    float o = 0.f, lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float wt = ex2_approx(sMw[w * G + h] - m_use);  // 0 for a warp that saw no key
+      o = fmaf(wt, red[(w * 32 + l) * kRow + h * DL + e], o);
+      lsum = fmaf(wt, sLw[w * G + h], lsum);
+    }
     if (p.n_split == 1) {
       const bool has = lsum > 0.f;
       const float v = has ? o / lsum : 0.f;
