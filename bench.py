@@ -66,7 +66,7 @@ BWD_NCU_TRAFFIC = {
 # The same for the decode kernel (mfa_decode_kernel) of --pass decode.
 DEC_KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/decode_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh")
 DEC_NCU_TRAFFIC = {
-    "decode_sel64k": (138_088_960, "9b364fe4d18fa820"),
+    "decode_sel64k": (141_120_000, "2b05ba268e1ffe33"),
 }
 
 
