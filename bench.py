@@ -233,7 +233,6 @@ def oracle_mask(mask):
 def run_reference(args, prob, pairs, d, Hq):
     """The reference arm: the float64 CPU oracle, each step a bounded sample of the workload."""
     from threadpoolctl import threadpool_info
-    from oracle import attention as OA
     heads = list(range(min(args.reference_heads, Hq)))
     flops = 4.0 * d * pairs * len(heads) / (1 if prob.mask.Hm == 1 else Hq)
     omask = oracle_mask(prob.mask)
@@ -247,7 +246,7 @@ def run_reference(args, prob, pairs, d, Hq):
         if args.pass_ == "bwd":
             OB.attention_backward(prob.q, prob.k, prob.v, omask, dout, heads=heads)
         else:
-            OA.attention(prob.q, prob.k, prob.v, omask, heads=heads)
+            oracle_forward(prob, omask, heads, args.bias, Hq)
         if s >= args.warmup:
             times.append(time.perf_counter() - t0)
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -258,7 +257,7 @@ def run_reference(args, prob, pairs, d, Hq):
         "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": args.workload, "pass": args.pass_,
+        "config": {"workload": args.workload, "pass": args.pass_, "bias": args.bias,
                    "sample": f"{len(heads)} of {Hq} query heads, all rows"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"{len(heads)} of {Hq} query heads, all rows, float64 numpy"},
@@ -266,13 +265,22 @@ def run_reference(args, prob, pairs, d, Hq):
     }
 
 
-def cpu_baseline(prob, pairs, d, Hq, heads_n):
+def oracle_forward(prob, omask, heads, bias, Hq):
+    """One oracle forward over the sampled heads, with the additive bias when one is named."""
+    if bias == "none":
+        from oracle import attention as OA
+        return OA.attention(prob.q, prob.k, prob.v, omask, heads=heads)
+    from oracle import bias as OBias
+    kind = {"alibi": OBias.LINEAR, "alibi_sqrt": OBias.SQRT, "alibi_left": OBias.LEFT}[bias]
+    return OBias.attention_bias(prob.q, prob.k, prob.v, omask, kind, OBias.alibi_slopes(Hq), heads=heads)
+
+
+def cpu_baseline(prob, pairs, d, Hq, heads_n, bias="none"):
     from threadpoolctl import threadpool_info
-    from oracle import attention as OA
     heads = list(range(min(heads_n, Hq)))
     omask = oracle_mask(prob.mask)
     t0 = time.perf_counter()
-    OA.attention(prob.q, prob.k, prob.v, omask, heads=heads)
+    oracle_forward(prob, omask, heads, bias, Hq)
     sec = time.perf_counter() - t0
     flops = 4.0 * d * pairs * len(heads) / (1 if prob.mask.Hm == 1 else Hq)
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -614,6 +622,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.bias != "none" and args.pass_ != "fwd":
+        raise SystemExit("--bias applies to the forward pass only")
     if args.pass_ == "decode":
         args.workload = args.workload or "decode_sel64k"
         if args.workload not in W.DECODE_WORKLOADS:
@@ -781,7 +791,7 @@ def main():
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline and world == 1:
-        res["cpu_baseline"] = cpu_baseline(prob, pairs, d, Hq, args.oracle_heads)
+        res["cpu_baseline"] = cpu_baseline(prob, pairs, d, Hq, args.oracle_heads, args.bias)
     print(json.dumps(res), flush=True)
 
 
