@@ -754,22 +754,9 @@ bool bwd_layout(int64_t B, int64_t Hq, int64_t Nq, int64_t D, int64_t nqt, int64
   return true;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn_bwd() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
 // bf16 [B, H, N, D] tensor, 64-column SW128 boxes of `rows` rows.
 bool map_bf16(CUtensorMap* map, const mfa_tensor* t, int rows) {
-  auto fn = encode_fn_bwd();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(t->D), static_cast<cuuint64_t>(t->N),
                         static_cast<cuuint64_t>(t->H), static_cast<cuuint64_t>(t->B)};
@@ -784,7 +771,7 @@ bool map_bf16(CUtensorMap* map, const mfa_tensor* t, int rows) {
 
 // The fp32 dQ accumulator [B, Hq, Nq, D] (contiguous), 32 rows x 128 columns per box, no swizzle.
 bool map_dq(CUtensorMap* map, void* base, int64_t B, int64_t Hq, int64_t Nq) {
-  auto fn = encode_fn_bwd();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(Nq), static_cast<cuuint64_t>(Hq),
                         static_cast<cuuint64_t>(B)};
@@ -811,13 +798,6 @@ mfa_status check_bf16(const mfa_tensor* t) {
 
 bool same_shape(const mfa_tensor* a, const mfa_tensor* b) {
   return a->B == b->B && a->H == b->H && a->N == b->N && a->D == b->D;
-}
-
-int sm_count_bwd() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
 }
 
 }  // namespace
@@ -922,20 +902,15 @@ extern "C" mfa_status mfa_bwd(const mfa_tensor* q, const mfa_tensor* k, const mf
     // first, which re-read them from DRAM). With few items per CTA the end of
     // the launch dominates and longest first balances it (doc8k: 10 % faster);
     // block-selection lists are scattered, so there only the balance counts.
-    const int sms_ = sm_count_bwd();
+    const int sms_ = device_sm_count();
     p.order_lpt = (mask->kind == MFA_MASK_BLOCKSEL || n_items64 < 8 * static_cast<int64_t>(sms_ > 0 ? sms_ : 148)) ? 1 : 0;
     p.dk = static_cast<__nv_bfloat16*>(dk->data); p.dks0 = dk->stride[0]; p.dks1 = dk->stride[1]; p.dks2 = dk->stride[2];
     p.dv = static_cast<__nv_bfloat16*>(dv->data); p.dvs0 = dv->stride[0]; p.dvs1 = dv->stride[1]; p.dvs2 = dv->stride[2];
     p.err = map->err;
     p.sched = words;
-    static bool attr_set = false;
-    if (!attr_set) {
-      if (cudaFuncSetAttribute(mfa_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-          cudaSuccess)
-        return MFA_ERR_CUDA;
-      attr_set = true;
-    }
-    const int sms = sm_count_bwd();
+    static std::atomic<uint64_t> attr_devs{0};
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(mfa_bwd_kernel), kSmemBytes, attr_devs)) return MFA_ERR_CUDA;
+    const int sms = device_sm_count();
     if (sms <= 0) return MFA_ERR_CUDA;
     const int grid = p.n_items < sms ? p.n_items : sms;
     mfa_bwd_kernel<<<grid, kThreads, kSmemBytes, s>>>(mq, mk, mv, mdo, mdq, lse2, delta, p);

@@ -464,21 +464,8 @@ __global__ void __launch_bounds__(kCombineThreads) mfa_decode_combine(const DecP
 // ------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn_dec() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
 bool map_kv(CUtensorMap* map, const mfa_tensor* t) {
-  auto fn = encode_fn_dec();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(t->D), static_cast<cuuint64_t>(t->N),
                         static_cast<cuuint64_t>(t->H), static_cast<cuuint64_t>(t->B)};
@@ -503,23 +490,12 @@ mfa_status check_dec_tensor(const mfa_tensor* t) {
   return MFA_OK;
 }
 
-int sm_count_dec() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
-}
-
 template <int D, int G>
 mfa_status launch_dec(const CUtensorMap& mk, const CUtensorMap& mv, const DecParams& p, cudaStream_t s) {
   using C = DecCfg<D>;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(mfa_decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kBytes) !=
-        cudaSuccess)
-      return MFA_ERR_CUDA;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr_devs{0};
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(mfa_decode_kernel<D, G>), C::kBytes, attr_devs))
+    return MFA_ERR_CUDA;
   const dim3 grid(p.n_split, p.Nq, p.B * p.Hkv);
   mfa_decode_kernel<D, G><<<grid, kWarpsFor<D, G> * 32, C::kBytes, s>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
@@ -548,7 +524,8 @@ mfa_status launch_dec_g(const CUtensorMap& mk, const CUtensorMap& mv, const DecP
 // output write, so fewer and longer parts are faster once the SMs are busy
 // (decode_sel64k: 2 parts 2.35 TB/s, 4 parts 1.99, 16 parts 1.28).
 int32_t auto_split(int64_t rows, int32_t sel_k, int D) {
-  const int sms = sm_count_dec() > 0 ? sm_count_dec() : 148;
+  const int n_sm = device_sm_count();
+  const int sms = n_sm > 0 ? n_sm : 148;
   const int bytes = D == 128 ? DecCfg<128>::kBytes : DecCfg<256>::kBytes;
   const int per_sm = (227 * 1024) / bytes > 0 ? (227 * 1024) / bytes : 1;
   const int64_t target = (static_cast<int64_t>(sms) * per_sm * 85 + 99) / 100;

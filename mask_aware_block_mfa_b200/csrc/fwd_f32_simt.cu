@@ -161,13 +161,9 @@ __global__ void __launch_bounds__(kRowsPerBlock) mfa_fwd_f32_kernel(const F32Par
 template <int D>
 mfa_status launch_d(const F32Params& p, cudaStream_t s) {
   const size_t smem = (kRowsPerBlock * (D + 1) + 2 * kChunk * D) * sizeof(float) + kChunk * sizeof(int4);
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(mfa_fwd_f32_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return MFA_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_devs{0};
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(mfa_fwd_f32_kernel<D>), static_cast<int>(smem), attr_devs))
+    return MFA_ERR_CUDA;
   const dim3 grid((p.Nq + kRowsPerBlock - 1) / kRowsPerBlock, p.Hq, p.B);
   mfa_fwd_f32_kernel<D><<<grid, kRowsPerBlock, smem, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;

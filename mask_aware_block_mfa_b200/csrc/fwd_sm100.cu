@@ -845,21 +845,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
 bool make_map(CUtensorMap* map, const mfa_tensor* t, int box_rows) {
-  auto fn = encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(t->D), static_cast<cuuint64_t>(t->N),
                         static_cast<cuuint64_t>(t->H), static_cast<cuuint64_t>(t->B)};
@@ -885,25 +872,14 @@ mfa_status check_tensor(const mfa_tensor* t) {
   return MFA_OK;
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
-}
-
 template <int D, int BK, int GP, int kBias>
 mfa_status launch_b(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
                     cudaStream_t s) {
   using C = Cfg<D, BK>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(mfa_fwd_kernel<D, BK, GP, kBias>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kAlloc) != cudaSuccess)
-      return MFA_ERR_CUDA;
-    attr_set = true;
-  }
-  const int sms = sm_count();
+  static std::atomic<uint64_t> attr_devs{0};
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(mfa_fwd_kernel<D, BK, GP, kBias>), C::kAlloc, attr_devs))
+    return MFA_ERR_CUDA;
+  const int sms = device_sm_count();
   if (sms <= 0) return MFA_ERR_CUDA;
   const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: at most one CTA per SM
   mfa_fwd_kernel<D, BK, GP, kBias><<<grid, kThreads, C::kAlloc, s>>>(mq, mk, mv, p);

@@ -1,8 +1,11 @@
 // Host-side helpers shared by the translation units of libmfa.so.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "mfa.h"
@@ -14,6 +17,44 @@ constexpr int kMaxSelK = 256;
 
 inline int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// The driver's cuTensorMapEncodeTiled (through the runtime, so the library
+// does not link libcuda), looked up on first use; nullptr if unavailable.
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::atomic<void*> cached{nullptr};
+  void* fn = cached.load(std::memory_order_acquire);
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return nullptr;
+    cached.store(fn, std::memory_order_release);
+  }
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+// Streaming multiprocessors of the current device (0 on error).
+inline int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// A kernel's dynamic shared-memory limit is a per-device attribute:
+// cudaFuncSetAttribute sets it for the current device only. `done` holds
+// one bit per device (0..63) on which it is already set, so that a process
+// driving several GPUs sets it once on each.
+inline bool ensure_smem_attr(const void* func, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t{1} << dev) : 0;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return true;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
 
 // Byte offsets of the tile map's arrays inside its device buffer.
 struct MapLayout {
