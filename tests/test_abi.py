@@ -291,3 +291,16 @@ def test_fwd_bias_rejects_bad_arguments_on_host(lib):
     mf = _fake_map(lib, bq=128)
     d = _fake_mask(mf)
     assert call(B.MfaBias(B.BIAS_ALIBI, 0, 0x7600_0000_0000), *f32) == B.MFA_ERR_UNSUPPORTED  # fp32 + bias
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without libmfa.so every entry of the binding raises: there is no fallback path."""
+    missing = str(tmp_path / "libmfa.so")
+    monkeypatch.setattr(B, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        B.load(missing)
+    monkeypatch.setattr(B.load, "__defaults__", (missing,))
+    with pytest.raises(RuntimeError, match="missing"):
+        B.status_string(0)
+    with pytest.raises(RuntimeError, match="missing"):
+        B.decode_workspace_bytes(1, 8, 2, 1, 256, 16)
