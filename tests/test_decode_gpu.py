@@ -101,3 +101,15 @@ def test_decode_full_size_workload():
     assert err == 0
     ref_out, ref_lse = OD.decode_attention(q[:2], k[:2], v[:2], sel[:2])
     compare_attention(out[:2], lse[:2], ref_out, ref_lse)
+
+
+def test_decode_longest_lists():
+    """Lists of the maximum length (256 entries, 16 pads and 16 duplicates) over
+    a cache of 20000 keys (313 blocks, ragged last block), with the automatic
+    split and with 3 parts."""
+    q, k, v, sel = _inputs(9, 2, 8, 2, 2, 20000, 256, 256, pads=16, dups=16)
+    ref = OD.decode_attention(q, k, v, sel)
+    for n_split in (0, 3):
+        out, lse, err = run(q, k, v, sel, n_split)
+        assert err == 0
+        compare_attention(out, lse, *ref)

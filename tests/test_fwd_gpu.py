@@ -203,3 +203,19 @@ def test_fwd_full_size_sampled(name, bq, bk):
     compare_attention(got_out, got_lse, ref_out, ref_lse)
     if name == "band16k_neg":   # 64 rows per (b, h) see no key
         assert torch.isneginf(lse[:, :, :64]).all() and torch.isfinite(lse[:, :, 64:]).all()
+
+
+def test_fwd_blocksel_longest_lists():
+    """Selection lists of the maximum length (256 entries per 64-query block),
+    uniform over all 266 key blocks of 17000 keys: -1 pads, duplicates and
+    entries above the diagonal (ignored), and a ragged last block."""
+    rng = np.random.default_rng(31)
+    mask = W.random_blocksel(rng, 1, 17000, 17000, 256, p_pad=0.3)
+    prob = small_problem(mask, 2, 1, 128, 31)
+    rows = sample_rows(17000, 64, np.random.default_rng(3))
+    ref_out, ref_lse = oracle_rows(prob, rows)
+    for bq, bk in ((64, 64), (128, 128)):
+        out, lse, arrays, err = run_gpu(prob, bq, bk)
+        assert err == 0
+        compare_map(arrays, mask, bq, bk)
+        compare_attention(out[:, :, rows], lse[:, :, rows], ref_out, ref_lse)
