@@ -436,12 +436,16 @@ __global__ void __launch_bounds__(kWarpsFor<D, G> * 32, 1)
 // Combine the n_split partials of every (batch, key/value head, row): with
 // M = max m_s, out = sum o_s 2^(m_s - M) / sum l_s 2^(m_s - M). All parts
 // empty gives M = -FLT_MAX, weights 1 on zeros, l = 0: out = 0, lse = -inf.
+// One thread per output element, grid (rows, ceil(G * D / kCombineThreads)):
+// every thread waits for two rounds of loads only (the parts' m, then their
+// o and l), and the rows' CTAs spread over all SMs.
 template <int D, int G>
 __global__ void __launch_bounds__(kCombineThreads) mfa_decode_combine(const DecParams p) {
   const size_t ru = blockIdx.x;  // (bg, i)
   const int bg = static_cast<int>(ru / p.Nq), i = static_cast<int>(ru % p.Nq);
   const int b = bg / p.Hkv, g = bg % p.Hkv;
-  for (int it = threadIdx.x; it < G * D; it += kCombineThreads) {
+  const int it = blockIdx.y * kCombineThreads + threadIdx.x;
+  if (it < G * D) {
     const int h = it / D, d = it % D;
     float M = -FLT_MAX;
     for (int s = 0; s < p.n_split; ++s) M = fmaxf(M, p.ml_part[((ru * p.n_split + s) * G + h) * 2]);
@@ -500,7 +504,8 @@ mfa_status launch_dec(const CUtensorMap& mk, const CUtensorMap& mv, const DecPar
   mfa_decode_kernel<D, G><<<grid, kWarpsFor<D, G> * 32, C::kBytes, s>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
   if (p.n_split > 1) {
-    mfa_decode_combine<D, G><<<static_cast<unsigned>(p.B * p.Hkv * p.Nq), kCombineThreads, 0, s>>>(p);
+    const dim3 cgrid(static_cast<unsigned>(p.B * p.Hkv * p.Nq), (G * D + kCombineThreads - 1) / kCombineThreads);
+    mfa_decode_combine<D, G><<<cgrid, kCombineThreads, 0, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
   }
   return MFA_OK;
@@ -572,6 +577,7 @@ extern "C" mfa_status mfa_decode(const mfa_tensor* q, const mfa_tensor* k, const
   if (sel_k > kMaxSelK || q->B * k->H > 65535 || q->N > 65535 || k->N > (int64_t(1) << 30))
     return MFA_ERR_UNSUPPORTED;
   const int64_t rows = q->B * k->H * q->N;
+  if (rows > 0x7fffffff) return MFA_ERR_UNSUPPORTED;  // the combine grid has one CTA column per row
   const int32_t ns = n_split == 0 ? auto_split(rows > 0 ? rows : 1, sel_k, static_cast<int>(q->D)) : n_split;
   if (ns > 65535) return MFA_ERR_UNSUPPORTED;
   if (ns > 1) {
