@@ -280,13 +280,30 @@ def oracle_forward(prob, omask, heads, bias, Hq):
     return OBias.attention_bias(prob.q, prob.k, prob.v, omask, kind, OBias.alibi_slopes(Hq), heads=heads)
 
 
+CPU_SAMPLE_S = 15.0  # oracle work per cpu_baseline sample
+
+
+def timed_sample(run_unit, n_units: int, fixed: int = 0, budget_s: float = CPU_SAMPLE_S):
+    """Run run_unit(0), run_unit(1), ... and time them: `fixed` units when it is
+    positive, else as many as fit about budget_s seconds (at least one, at most
+    n_units). Returns (units run, seconds)."""
+    limit = min(fixed, n_units) if fixed > 0 else n_units
+    done, total = 0, 0.0
+    while done < limit:
+        t0 = time.perf_counter()
+        run_unit(done)
+        total += time.perf_counter() - t0
+        done += 1
+        if fixed <= 0 and total + total / done > budget_s:
+            break
+    return done, total
+
+
 def cpu_baseline(prob, pairs, d, Hq, heads_n, bias="none"):
     from threadpoolctl import threadpool_info
-    heads = list(range(min(heads_n, Hq)))
     omask = oracle_mask(prob.mask)
-    t0 = time.perf_counter()
-    oracle_forward(prob, omask, heads, bias, Hq)
-    sec = time.perf_counter() - t0
+    n, sec = timed_sample(lambda h: oracle_forward(prob, omask, [h], bias, Hq), Hq, heads_n)
+    heads = list(range(n))
     flops = 4.0 * d * pairs * len(heads) / (1 if prob.mask.Hm == 1 else Hq)
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     return {"value": flops / sec / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -422,11 +439,10 @@ def run_backward(args, prob, pairs, rank, world, local):
     if not args.no_cpu_baseline and world == 1:
         from threadpoolctl import threadpool_info
         from oracle import backward as OB
-        heads = list(range(min(args.oracle_heads, Hq)))
-        t0 = time.perf_counter()
-        OB.attention_backward(prob.q, prob.k, prob.v, oracle_mask(prob.mask), bwd_output_gradient(prob),
-                              heads=heads)
-        sec = time.perf_counter() - t0
+        omask, dout = oracle_mask(prob.mask), bwd_output_gradient(prob)
+        n, sec = timed_sample(lambda h: OB.attention_backward(prob.q, prob.k, prob.v, omask, dout, heads=[h]),
+                              Hq, args.oracle_heads)
+        heads = list(range(n))
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
         res["cpu_baseline"] = {"value": 10.0 * d * pairs * len(heads) / sec / 1e12, "unit": "TFLOP/s",
                                "cores": threads, "kind": "oracle",
@@ -595,12 +611,12 @@ def run_decode(args, rank, world, local):
     }
     if not args.no_cpu_baseline and world == 1:
         from oracle import decode as OD
-        t0 = time.perf_counter()
-        OD.decode_attention(q[:1], k[:1], v[:1], sel[:1])
-        sec = time.perf_counter() - t0
+        n, sec = timed_sample(lambda b: OD.decode_attention(q[b:b + 1], k[b:b + 1], v[b:b + 1], sel[b:b + 1]), B_,
+                              args.oracle_heads)
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-        res["cpu_baseline"] = {"value": nbytes / B_ / sec / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                               "sample": f"1 of {B_} sequences, float64 numpy ({sec:.1f} s)"}
+        res["cpu_baseline"] = {"value": nbytes * n / B_ / sec / 1e9, "unit": "GB/s", "cores": threads,
+                               "kind": "oracle",
+                               "sample": f"{n} of {B_} sequences, float64 numpy ({sec:.1f} s)"}
     print(json.dumps(res), flush=True)
 
 
@@ -611,7 +627,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=None, choices=sorted(BLOCKS) + sorted(W.DECODE_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--oracle-heads", type=int, default=4, help="query heads in the CPU-baseline sample")
+    ap.add_argument("--oracle-heads", type=int, default=0,
+                    help="units (query heads; sequences for decode) in the CPU-baseline sample; "
+                         "0 = as many as fit about 15 s")
     ap.add_argument("--reference-heads", type=int, default=1, help="query heads per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)

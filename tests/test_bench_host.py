@@ -74,3 +74,22 @@ def test_decode_bytes_count_the_oracle_visibility():
     keys = sum(int(OD.visible_dense(sel, b, g, 3, 1000).sum()) for b in range(2) for g in range(2))
     expect = keys * 128 * 2 * 2 + 2 * q.numel() * 2 + 2 * 8 * 3 * 4 + sel.size * 4
     assert bench.decode_bytes(q, k, sel) == expect
+
+
+def test_cpu_sample_sizing(monkeypatch):
+    """timed_sample: a fixed count when asked, else units until the next would
+    pass the budget (at least one, at most all)."""
+    import bench
+    clock = [0.0]
+    monkeypatch.setattr(bench.time, "perf_counter", lambda: clock[0])
+
+    def unit(cost):
+        def run(_):
+            clock[0] += cost
+        return run
+
+    assert bench.timed_sample(unit(1.0), 32, fixed=4) == (4, 4.0)
+    assert bench.timed_sample(unit(1.0), 3, fixed=10) == (3, 3.0)
+    assert bench.timed_sample(unit(4.0), 32, budget_s=15.0) == (3, 12.0)   # a fourth would reach 16 s
+    assert bench.timed_sample(unit(40.0), 32, budget_s=15.0) == (1, 40.0)  # one unit even above the budget
+    assert bench.timed_sample(unit(0.1), 5, budget_s=15.0)[0] == 5         # never more than all units
