@@ -136,7 +136,44 @@ def _check(fn: str, code: int) -> None:
         raise MfaError(fn, code, status_string(code))
 
 
-def tensor_desc(t: torch.Tensor) -> MfaTensor:
+def _on_device(name: str, t, device=None, dtype=None, shape=None, contiguous=False) -> None:
+    """Host-side checks of a tensor handed to the library as a raw device
+    pointer: a CUDA tensor, on `device` when given, with the dtype, shape and
+    layout the call reads or writes (the C ABI cannot check these for plain
+    pointers, and a host pointer would fault the kernel)."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call runs on {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check_lse(lse, q) -> None:
+    _on_device("lse", lse, q.device, torch.float32, tuple(q.shape[:3]), contiguous=True)
+
+
+def _dev(q):
+    """The device of the call (q's), after checking that q is a CUDA tensor."""
+    _on_device("q", q)
+    return q.device
+
+
+def _same_device(q, *holders) -> None:
+    """The device arrays of masks and tile maps must live on q's device."""
+    for h in holders:
+        ts = [getattr(h, "buf", None), getattr(h, "bounds", None)] + list(getattr(h, "_keep", []))
+        for t in ts:
+            if isinstance(t, torch.Tensor) and t.device != q.device:
+                raise ValueError(f"a mask or tile-map array is on {t.device}, q on {q.device}")
+
+
+def tensor_desc(t: torch.Tensor, device=None) -> MfaTensor:
+    _on_device("tensor", t, device)
     if t.dim() != 4:
         raise ValueError("expected a [B, H, N, D] tensor")
     dt = {torch.bfloat16: MFA_BF16, torch.float32: MFA_F32}.get(t.dtype)
@@ -262,10 +299,10 @@ def build_tile_map(dmask: DeviceMask, tmap: TileMap, stream=None) -> None:
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: DeviceMask, tmap: TileMap,
         out: torch.Tensor, lse: torch.Tensor, stream=None) -> None:
     """out, lse <- attention(q, k, v) under dmask, through the tile map (both on the device)."""
-    if lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 tensor")
+    qd, kd, vd, od = (tensor_desc(t, _dev(q)) for t in (q, k, v, out))
+    _check_lse(lse, q)
+    _same_device(q, tmap, dmask)
     dmask.desc.map = ctypes.pointer(tmap.m)
-    qd, kd, vd, od = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
     _check("mfa_fwd", load().mfa_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(dmask.desc),
                                      ctypes.byref(od), lse.data_ptr(), _stream_ptr(stream)))
 
@@ -273,13 +310,12 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: DeviceMask, tm
 def fwd_bias(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask, tmap: TileMap, kind: int,
              slopes: torch.Tensor, out: torch.Tensor, lse: torch.Tensor, stream=None) -> None:
     """Forward pass with an additive ALiBi bias (kind BIAS_*, slopes: float32 device tensor [Hq])."""
-    if lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 tensor")
-    if slopes.dtype != torch.float32 or not slopes.is_contiguous():
-        raise ValueError("slopes must be a contiguous float32 tensor")
+    qd, kd, vd, od = (tensor_desc(t, _dev(q)) for t in (q, k, v, out))
+    _check_lse(lse, q)
+    _on_device("slopes", slopes, q.device, torch.float32, (int(q.shape[1]),), contiguous=True)
+    _same_device(q, tmap, dmask)
     dmask.desc.map = ctypes.pointer(tmap.m)
     bias = MfaBias(kind, 0, slopes.data_ptr())
-    qd, kd, vd, od = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
     _check("mfa_fwd_bias", load().mfa_fwd_bias(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd),
                                                ctypes.byref(dmask.desc), ctypes.byref(bias), ctypes.byref(od),
                                                lse.data_ptr(), _stream_ptr(stream)))
@@ -288,9 +324,13 @@ def fwd_bias(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask, tmap: Til
 def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: DeviceMask, block_q: int, block_k: int,
                 out: torch.Tensor, lse: torch.Tensor, dev_err: Optional[torch.Tensor] = None, stream=None) -> None:
     """Forward pass with the tile map in the library's own device array (no allocation by anyone)."""
-    if lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 tensor")
-    qd, kd, vd, od = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
+    qd, kd, vd, od = (tensor_desc(t, _dev(q)) for t in (q, k, v, out))
+    _check_lse(lse, q)
+    if dev_err is not None:
+        _on_device("dev_err", dev_err, q.device)
+        if dev_err.numel() * dev_err.element_size() < 4:
+            raise ValueError("dev_err must hold at least 4 bytes")
+    _same_device(q, dmask)
     err_ptr = None if dev_err is None else dev_err.data_ptr()
     _check("mfa_fwd_noalloc", load().mfa_fwd_noalloc(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd),
                                                      ctypes.byref(dmask.desc), block_q, block_k, ctypes.byref(od),
@@ -305,12 +345,11 @@ def bwd(q, k, v, out, dout, lse, dmask, tmap: TileMap, dq, dk, dv, workspace: to
     """dq, dk, dv <- gradients of attention(q, k, v) under dmask for the output
     gradient dout (out, lse from the forward pass; the map built with 128-key
     tiles); workspace is a uint8 device tensor of bwd_workspace_bytes()."""
-    if lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 tensor")
-    if workspace.dtype != torch.uint8 or not workspace.is_contiguous():
-        raise ValueError("workspace must be a contiguous uint8 tensor")
+    ds = [tensor_desc(t, _dev(q)) for t in (q, k, v, out, dout, dq, dk, dv)]
+    _check_lse(lse, q)
+    _on_device("workspace", workspace, q.device, torch.uint8, contiguous=True)
+    _same_device(q, tmap, dmask)
     dmask.desc.map = ctypes.pointer(tmap.m)
-    ds = [tensor_desc(t) for t in (q, k, v, out, dout, dq, dk, dv)]
     _check("mfa_bwd", load().mfa_bwd(*(ctypes.byref(d) for d in ds[:5]), lse.data_ptr(), ctypes.byref(dmask.desc),
                                      *(ctypes.byref(d) for d in ds[5:]), workspace.data_ptr(), workspace.numel(),
                                      _stream_ptr(stream)))
@@ -331,11 +370,13 @@ class Decode:
 
     def __call__(self, q, k, v, sel, out=None, lse=None, stream=None):
         """sel: int32 device tensor [B, Hkv, Nq, sel_k] of 64-key block indices (-1 = none)."""
-        if sel.dtype != torch.int32 or not sel.is_contiguous() or sel.dim() != 4:
-            raise ValueError("sel must be a contiguous int32 [B, Hkv, Nq, sel_k] tensor")
+        qd, kd, vd = (tensor_desc(t, _dev(q)) for t in (q, k, v))
         B_, Hq, Nq, D = q.shape
         Hkv = int(k.shape[1])
+        if sel.dim() != 4:
+            raise ValueError("sel must be a [B, Hkv, Nq, sel_k] tensor")
         sel_k = int(sel.shape[-1])
+        _on_device("sel", sel, q.device, torch.int32, (B_, Hkv, Nq, sel_k), contiguous=True)
         need = decode_workspace_bytes(B_, Hq, Hkv, Nq, D, sel_k, self.n_split)
         if need == 0:
             raise ValueError("invalid decode sizes")
@@ -345,7 +386,8 @@ class Decode:
             self.err = torch.zeros(1, dtype=torch.int32, device=q.device)
         out = torch.empty_like(q) if out is None else out
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if lse is None else lse
-        qd, kd, vd, od = tensor_desc(q), tensor_desc(k), tensor_desc(v), tensor_desc(out)
+        od = tensor_desc(out, q.device)
+        _check_lse(lse, q)
         _check("mfa_decode", load().mfa_decode(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), sel.data_ptr(),
                                                sel_k, ctypes.byref(od), lse.data_ptr(), self.n_split,
                                                self.ws.data_ptr(), self.ws.numel(), self.err.data_ptr(),

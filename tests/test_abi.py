@@ -304,3 +304,22 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
         B.status_string(0)
     with pytest.raises(RuntimeError, match="missing"):
         B.decode_workspace_bytes(1, 8, 2, 1, 256, 16)
+
+
+def test_binding_rejects_host_tensors():
+    """A host tensor never reaches a kernel as a pointer: every wrapper raises first."""
+    import torch
+    q = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 2, 8)
+    ws = torch.zeros(16, dtype=torch.uint8)
+    calls = [
+        lambda: B.fwd(q, q, q, None, None, q, lse),
+        lambda: B.fwd_bias(q, q, q, None, None, B.BIAS_ALIBI, torch.zeros(2), q, lse),
+        lambda: B.fwd_noalloc(q, q, q, None, 64, 128, q, lse),
+        lambda: B.bwd(q, q, q, q, q, lse, None, None, q, q, q, ws),
+        lambda: B.Decode()(q, q, q, torch.zeros(1, 2, 8, 4, dtype=torch.int32)),
+        lambda: B.tensor_desc(q),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()

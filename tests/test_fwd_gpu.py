@@ -219,3 +219,25 @@ def test_fwd_blocksel_longest_lists():
         assert err == 0
         compare_map(arrays, mask, bq, bk)
         compare_attention(out[:, :, rows], lse[:, :, rows], ref_out, ref_lse)
+
+
+def test_binding_checks_raw_pointer_arguments():
+    """Arguments passed as plain device pointers (lse, slopes, selection lists)
+    are checked for dtype and shape before the call: a short buffer would be
+    written past its end."""
+    mask = W.band(1, 256, 64, 0)
+    prob = small_problem(mask, 2, 1, 128, 4)
+    att = B.Attention(mask, 128, 128)
+    att.build()
+    q, k, v = (t.cuda() for t in (prob.q, prob.k, prob.v))
+    with pytest.raises(ValueError, match="lse"):
+        att(q, k, v, lse=torch.empty(1, 2, 255, device="cuda"))
+    with pytest.raises(ValueError, match="lse"):
+        att(q, k, v, lse=torch.empty(1, 2, 256, dtype=torch.float64, device="cuda"))
+    with pytest.raises(ValueError, match="slopes"):
+        att(q, k, v, bias=(B.BIAS_ALIBI, torch.ones(1, device="cuda")))
+    dec = B.Decode()
+    with pytest.raises(ValueError, match="sel"):
+        dec(q[:, :, :1], k, v, torch.zeros(1, 2, 1, 4, dtype=torch.int32, device="cuda"))  # Hkv is 1, not 2
+    out, lse = att(q, k, v)
+    assert B.device_status(att.tmap) == 0 and torch.isfinite(lse).all()
