@@ -345,7 +345,8 @@ size_t mfa_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t Nq
  *   listed and j <= i + Nk - Nq (with Nq == Nk, the rule of MFA_MASK_BLOCKSEL).
  *   Rows that see no key get out = 0 and lse = -inf.
  *   lse     float32 [B, Hq, Nq] contiguous, natural log.
- *   n_split parts per list (0 = chosen for at least two CTAs per SM); with
+ *   n_split parts per list (0 = the fewest parts whose CTAs fill at least
+ *           85 % of one wave on the SMs, at most sel_k / 2); with
  *           n_split > 1 the parts are combined by a second kernel (empty parts
  *           carry m = -FLT_MAX, so no exp(-inf - -inf) arises) and `workspace`
  *           (DEVICE, 256-byte aligned, mfa_decode_workspace_bytes bytes, owned
