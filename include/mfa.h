@@ -17,13 +17,20 @@
  *                       calculations for fully masked blocks are unnecessary).
  *   mfa_bwd             computes dq, dk, dv through the same map (FlashMask's
  *                       masks serve training first, per the author response).
+ *   mfa_decode          attends a few query rows to selected 64-key blocks of a
+ *                       long cache, split over CTAs (the selected-key flash
+ *                       attention pull request).
+ * mfa_fwd_bias adds an ALiBi bias to mfa_fwd, mfa_mask_from_sparse_mode turns
+ * an Ascend sparse mode into a mask description, and mfa_fwd_noalloc runs the
+ * map build and forward pass without any buffer from the caller but the tensors.
  *
  * Conventions shared by every call:
  *
  * - All tensor and array pointers are DEVICE pointers unless a comment says
  *   otherwise. The caller allocates and owns every buffer; the library
- *   allocates no device memory and keeps no state between calls except a
- *   per-process cache of kernel attributes.
+ *   allocates no device memory. Between calls it keeps only the record of
+ *   the devices on which it has set each kernel's shared-memory attribute,
+ *   and mfa_fwd_noalloc's static scratch array (part of the module).
  * - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
  *   is the legacy default stream). Argument errors are detected on the host and
  *   returned before anything is launched. Problems only the device can see
@@ -268,7 +275,7 @@ mfa_status mfa_fwd_bias(const mfa_tensor* q, const mfa_tensor* k, const mfa_tens
 /* The forward pass for callers that cannot allocate device memory: for
  * example a plugin inside a host application that owns the GPU allocator and
  * passes in only the tensors, or code that must not allocate at this point of
- * its pipeline. The paper has no counterpart; this is a convenience of the
+ * its pipeline. The pages have no counterpart; this is a convenience of the
  * library. It does what mfa_build_tile_map followed by mfa_fwd do, but the
  * tile map (block_q x block_k, each 64 or 128) and the forward pass's work
  * counters live in a fixed array of MFA_NOALLOC_SCRATCH_BYTES that the library
