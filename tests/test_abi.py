@@ -323,3 +323,19 @@ def test_binding_rejects_host_tensors():
     for call in calls:
         with pytest.raises(ValueError, match="CUDA tensor"):
             call()
+
+
+def test_mask_and_map_arrays_must_share_the_call_device():
+    """_same_device compares every device array a mask or map holds with q's device."""
+    import torch
+
+    class Holder:
+        pass
+
+    q = torch.zeros(1, 1, 4, 8)
+    same, other = Holder(), Holder()
+    same.buf, same._keep = torch.zeros(4), [torch.zeros(2)]
+    other.bounds = torch.empty(4, device="meta")
+    B._same_device(q, same)
+    with pytest.raises(ValueError, match="mask or tile-map array"):
+        B._same_device(q, same, other)
