@@ -7,7 +7,7 @@ each, over the whole job (all ranks). Inputs are seeded N(0,1) bf16 tensors of
 the named workload's shape; they are resident in HBM when timing starts, and L2
 is flushed (a 256 MiB write) between timed steps.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload doc8k] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload doc32k] [--impl ours|reference]
 
 Multi-GPU: one process per GPU (torchrun); each rank runs an independent
 replica of the workload (the path needs no exchange), so scaling is weak and
@@ -44,6 +44,11 @@ BLOCKS = {  # launch configuration per workload: (block_q, block_k)
     "varlen_prefill16k": (64, 128),
 }
 METRIC = "effective TFLOP/s (visible pairs only) and % of B200 bf16 tensor peak"
+# The default line times the largest single-GPU workload (32K tokens, causal
+# documents); the two document-mask workloads that carry the >= 50 % target
+# (8K and 32K) are also timed forward-only in the same run ("targets").
+DEFAULT_WORKLOAD = "doc32k"
+TARGET_WORKLOADS = ("doc8k", "doc32k")
 
 # DRAM bytes (read + write) of one forward launch, from one ncu capture of
 # the forward kernel on that workload (the summaries under profiles/ give the
@@ -620,6 +625,54 @@ def run_decode(args, rank, world, local):
     print(json.dumps(res), flush=True)
 
 
+def time_target(name: str, dev, stream, flush, steps: int, warmup: int) -> dict:
+    """Forward-only and map + forward times of a target workload (CUDA graphs,
+    L2 flushed between replays), with its effective TFLOP/s and fraction of
+    the measured burst bf16 peak."""
+    from mask_aware_block_mfa_b200 import binding as B
+    prob = W.make_problem(name)
+    _, Hq, _, _, d = prob.shape
+    flops = 4.0 * d * visible_pairs(prob.mask) * (Hq if prob.mask.Hm == 1 else 1)
+    bq, bk = BLOCKS[name]
+    q, k, v = (t.to(dev) for t in (prob.q, prob.k, prob.v))
+    att = B.Attention(B.DeviceMask(prob.mask, dev), bq, bk, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        att.build()
+        att(q, k, v, out, lse)
+    torch.cuda.synchronize(dev)
+    g_step, g_fwd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g_step, stream=cap):
+            att.build()
+            att(q, k, v, out, lse)
+        with torch.cuda.graph(g_fwd, stream=cap):
+            att(q, k, v, out, lse)
+    stream.wait_stream(cap)
+    for _ in range(warmup):
+        g_step.replay()
+        g_fwd.replay()
+    times = {}
+    for key, graph in (("step", g_step), ("fwd", g_fwd)):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for e0, e1 in evs:
+            flush.fill_(1.0)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        times[key] = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
+    if B.device_status(att.tmap, stream) != 0:
+        raise RuntimeError(f"device error word set while timing {name}")
+    burst, _, src = peaks()
+    tf = flops / (times["fwd"] * 1e-3) / 1e12
+    return {"fwd_ms": times["fwd"], "fwd_tflops": tf, "frac": tf / burst, "step_ms": times["step"],
+            "step_tflops": flops / (times["step"] * 1e-3) / 1e12, "peak": burst, "peaks": src}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -632,6 +685,8 @@ def main():
                          "0 = as many as fit about 15 s")
     ap.add_argument("--reference-heads", type=int, default=1, help="query heads per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-targets", action="store_true",
+                    help="skip the forward-only timing of the 8K and 32K document-mask workloads")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--bias", default="none", choices=["none", "alibi", "alibi_sqrt", "alibi_left"],
                     help="additive ALiBi bias in the forward pass (slopes 2^(-8h/Hq))")
@@ -652,7 +707,7 @@ def main():
         if args.workload not in W.DECODE_WORKLOADS:
             raise SystemExit("--pass decode takes a decode workload")
         return run_decode(args, rank, world, local)
-    args.workload = args.workload or "doc8k"
+    args.workload = args.workload or DEFAULT_WORKLOAD
     if args.workload not in BLOCKS:
         raise SystemExit("decode workloads run with --pass decode")
 
@@ -786,6 +841,19 @@ def main():
             e2e_ms.append(a.elapsed_time(z))
     e2e_value = flops * world / (statistics.mean(e2e_ms) * 1e-3) / 1e12
 
+    # The target workloads' forward-only figures (the main workload's from the
+    # timing above, the other's timed here), on every rank alike.
+    targets = {}
+    if not args.no_targets and args.bias == "none":
+        for name in TARGET_WORKLOADS:
+            if name == args.workload:
+                burst_t, _, src_t = peaks()
+                targets[name] = {"fwd_ms": fwd_avg_ms, "fwd_tflops": achieved, "frac": achieved / burst_t,
+                                 "step_ms": ms_per_step, "step_tflops": flops / (ms_per_step * 1e-3) / 1e12,
+                                 "peak": burst_t, "peaks": src_t}
+            else:
+                targets[name] = time_target(name, dev, stream, flush, args.steps, args.warmup)
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -815,6 +883,8 @@ def main():
         "gpu_launches": (4 if sparse and prob.mask.mode >= 5 else 3) * args.steps,
         "clocks": clk.summary(),
     }
+    if targets:
+        res["targets"] = targets
     if not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(prob, pairs, d, Hq, args.oracle_heads, args.bias)
     print(json.dumps(res), flush=True)

@@ -31,6 +31,9 @@
  *   allocates no device memory. Between calls it keeps only the record of
  *   the devices on which it has set each kernel's shared-memory attribute,
  *   and mfa_fwd_noalloc's static scratch array (part of the module).
+ * - Every call launches on the CURRENT CUDA device (cudaSetDevice), which must
+ *   be the device that holds the call's tensors and arrays, and `stream` must
+ *   belong to that device. The library does not switch devices itself.
  * - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
  *   is the legacy default stream). Argument errors are detected on the host and
  *   returned before anything is launched. Problems only the device can see
@@ -281,13 +284,18 @@ mfa_status mfa_fwd_bias(const mfa_tensor* q, const mfa_tensor* k, const mfa_tens
  * counters live in a fixed array of MFA_NOALLOC_SCRATCH_BYTES that the library
  * itself holds in device memory; nothing is allocated by anyone. mask->map is
  * ignored. q, k, v, out and lse are as for mfa_fwd.
- * - A map larger than MFA_NOALLOC_SCRATCH_BYTES (mfa_tile_map_bytes) returns
- *   MFA_ERR_UNSUPPORTED before anything is launched.
+ * - Every argument is checked on the host first, as mfa_fwd checks it; a map
+ *   larger than MFA_NOALLOC_SCRATCH_BYTES (mfa_tile_map_bytes) returns
+ *   MFA_ERR_UNSUPPORTED. A rejected call launches nothing and leaves the
+ *   array as it was.
  * - dev_err: optional DEVICE pointer to one uint32; after the pass it receives
  *   the device error bits (MFA_DEVERR_*) by a device-to-device copy on
  *   `stream`. NULL skips the copy.
- * - The first call on each device looks up the array's device address with
- *   that device current; make that first call before any stream capture.
+ * - The array's device address is looked up (cudaGetSymbolAddress) with the
+ *   call's device current: on the first call on each device, and again on
+ *   every later call made while `stream` is not capturing, so a
+ *   cudaDeviceReset between calls leaves no stale address behind. Make the
+ *   first call on each device before any stream capture.
  * - Every call on a device shares the one array and leaves its contents in it
  *   (each call clears and rebuilds what it uses). Calls that overlap on the
  *   GPU race: order them (one stream, or events between streams). */

@@ -188,10 +188,23 @@ def tensor_desc(t: torch.Tensor, device=None) -> MfaTensor:
     return d
 
 
-def _stream_ptr(stream) -> int:
+def _stream_ptr(stream, device=None) -> int:
+    """The raw handle of `stream`, by default the current stream of `device`.
+    A stream of another device is rejected: the library launches on the
+    current device, which every wrapper below sets to the tensors' device."""
+    if device is not None:
+        device = torch.device(device)
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and device.type == "cuda" and stream.device != device:
+        raise ValueError(f"the stream is on {stream.device}, the call runs on {device}")
     return int(stream.cuda_stream)
+
+
+def _on(device):
+    """Make `device` current for the duration of one library call (the C ABI
+    launches on the current device and looks up per-device state there)."""
+    return torch.cuda.device(torch.device(device))
 
 
 class DeviceMask:
@@ -249,9 +262,11 @@ class SparseModeMask:
         """(Re)write the description, and for modes 5-8 the bounds, from the
         mode's inputs already on the device (no allocation, graph-capturable)."""
         ptrs = [self.bounds[i].data_ptr() for i in range(4)]  # lts, lte, uts, ute
-        _check("mfa_mask_from_sparse_mode",
-               load().mfa_mask_from_sparse_mode(ctypes.byref(self.sm), self.B, self.Nq, self.Nk, *ptrs,
-                                                ctypes.byref(self.desc), _stream_ptr(stream)))
+        dev = self.bounds.device
+        with _on(dev):
+            _check("mfa_mask_from_sparse_mode",
+                   load().mfa_mask_from_sparse_mode(ctypes.byref(self.sm), self.B, self.Nq, self.Nk, *ptrs,
+                                                    ctypes.byref(self.desc), _stream_ptr(stream, dev)))
 
 
 class TileMap:
@@ -292,8 +307,11 @@ class TileMap:
 
 
 def build_tile_map(dmask: DeviceMask, tmap: TileMap, stream=None) -> None:
-    _check("mfa_build_tile_map", load().mfa_build_tile_map(ctypes.byref(dmask.desc), ctypes.byref(tmap.m),
-                                                           _stream_ptr(stream)))
+    dev = tmap.buf.device
+    _same_device(tmap.buf, dmask)
+    with _on(dev):
+        _check("mfa_build_tile_map", load().mfa_build_tile_map(ctypes.byref(dmask.desc), ctypes.byref(tmap.m),
+                                                               _stream_ptr(stream, dev)))
 
 
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: DeviceMask, tmap: TileMap,
@@ -303,8 +321,10 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: DeviceMask, tm
     _check_lse(lse, q)
     _same_device(q, tmap, dmask)
     dmask.desc.map = ctypes.pointer(tmap.m)
-    _check("mfa_fwd", load().mfa_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), ctypes.byref(dmask.desc),
-                                     ctypes.byref(od), lse.data_ptr(), _stream_ptr(stream)))
+    with _on(q.device):
+        _check("mfa_fwd", load().mfa_fwd(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd),
+                                         ctypes.byref(dmask.desc), ctypes.byref(od), lse.data_ptr(),
+                                         _stream_ptr(stream, q.device)))
 
 
 def fwd_bias(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask, tmap: TileMap, kind: int,
@@ -316,9 +336,10 @@ def fwd_bias(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask, tmap: Til
     _same_device(q, tmap, dmask)
     dmask.desc.map = ctypes.pointer(tmap.m)
     bias = MfaBias(kind, 0, slopes.data_ptr())
-    _check("mfa_fwd_bias", load().mfa_fwd_bias(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd),
-                                               ctypes.byref(dmask.desc), ctypes.byref(bias), ctypes.byref(od),
-                                               lse.data_ptr(), _stream_ptr(stream)))
+    with _on(q.device):
+        _check("mfa_fwd_bias", load().mfa_fwd_bias(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd),
+                                                   ctypes.byref(dmask.desc), ctypes.byref(bias), ctypes.byref(od),
+                                                   lse.data_ptr(), _stream_ptr(stream, q.device)))
 
 
 def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: DeviceMask, block_q: int, block_k: int,
@@ -332,9 +353,12 @@ def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dmask: Device
             raise ValueError("dev_err must hold at least 4 bytes")
     _same_device(q, dmask)
     err_ptr = None if dev_err is None else dev_err.data_ptr()
-    _check("mfa_fwd_noalloc", load().mfa_fwd_noalloc(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd),
-                                                     ctypes.byref(dmask.desc), block_q, block_k, ctypes.byref(od),
-                                                     lse.data_ptr(), err_ptr, _stream_ptr(stream)))
+    # The library picks its scratch array and launches on the current device.
+    with _on(q.device):
+        _check("mfa_fwd_noalloc", load().mfa_fwd_noalloc(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd),
+                                                         ctypes.byref(dmask.desc), block_q, block_k,
+                                                         ctypes.byref(od), lse.data_ptr(), err_ptr,
+                                                         _stream_ptr(stream, q.device)))
 
 
 def bwd_workspace_bytes(B: int, Hq: int, Nq: int, Nk: int, D: int) -> int:
@@ -350,9 +374,10 @@ def bwd(q, k, v, out, dout, lse, dmask, tmap: TileMap, dq, dk, dv, workspace: to
     _on_device("workspace", workspace, q.device, torch.uint8, contiguous=True)
     _same_device(q, tmap, dmask)
     dmask.desc.map = ctypes.pointer(tmap.m)
-    _check("mfa_bwd", load().mfa_bwd(*(ctypes.byref(d) for d in ds[:5]), lse.data_ptr(), ctypes.byref(dmask.desc),
-                                     *(ctypes.byref(d) for d in ds[5:]), workspace.data_ptr(), workspace.numel(),
-                                     _stream_ptr(stream)))
+    with _on(q.device):
+        _check("mfa_bwd", load().mfa_bwd(*(ctypes.byref(d) for d in ds[:5]), lse.data_ptr(),
+                                         ctypes.byref(dmask.desc), *(ctypes.byref(d) for d in ds[5:]),
+                                         workspace.data_ptr(), workspace.numel(), _stream_ptr(stream, q.device)))
 
 
 def decode_workspace_bytes(B: int, Hq: int, Hkv: int, Nq: int, D: int, sel_k: int, n_split: int = 0) -> int:
@@ -388,10 +413,11 @@ class Decode:
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if lse is None else lse
         od = tensor_desc(out, q.device)
         _check_lse(lse, q)
-        _check("mfa_decode", load().mfa_decode(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd), sel.data_ptr(),
-                                               sel_k, ctypes.byref(od), lse.data_ptr(), self.n_split,
-                                               self.ws.data_ptr(), self.ws.numel(), self.err.data_ptr(),
-                                               _stream_ptr(stream)))
+        with _on(q.device):
+            _check("mfa_decode", load().mfa_decode(ctypes.byref(qd), ctypes.byref(kd), ctypes.byref(vd),
+                                                   sel.data_ptr(), sel_k, ctypes.byref(od), lse.data_ptr(),
+                                                   self.n_split, self.ws.data_ptr(), self.ws.numel(),
+                                                   self.err.data_ptr(), _stream_ptr(stream, q.device)))
         return out, lse
 
     def status(self) -> int:
@@ -403,7 +429,9 @@ class Decode:
 def device_status(tmap: TileMap, stream=None) -> int:
     """Synchronise and return the map's device error bits (0 = none)."""
     bits = ctypes.c_uint32(0)
-    code = load().mfa_get_device_status(ctypes.byref(tmap.m), _stream_ptr(stream), ctypes.byref(bits))
+    dev = tmap.buf.device
+    with _on(dev):
+        code = load().mfa_get_device_status(ctypes.byref(tmap.m), _stream_ptr(stream, dev), ctypes.byref(bits))
     if code not in (MFA_OK, MFA_ERR_DEVICE):
         _check("mfa_get_device_status", code)
     return int(bits.value)

@@ -917,9 +917,9 @@ extern "C" mfa_status mfa_fwd_bias(const mfa_tensor* q, const mfa_tensor* k, con
 }
 
 namespace mfa {
-namespace {
-mfa_status fwd_impl(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v, const mfa_mask_desc* mask,
-                    const mfa_bias* bias, const mfa_tensor* out, float* lse, void* stream) {
+
+mfa_status check_fwd_args(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v, const mfa_mask_desc* mask,
+                          const mfa_bias* bias, const mfa_tensor* out, const float* lse, int32_t block_q) {
   mfa_status st;
   const int32_t bias_kind = bias ? bias->kind : MFA_BIAS_NONE;
   if (bias_kind < MFA_BIAS_NONE || bias_kind > MFA_BIAS_ALIBI_LEFT) return MFA_ERR_INVALID_ARG;
@@ -929,10 +929,6 @@ mfa_status fwd_impl(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* 
     return st;
   if (!lse && q->N > 0) return MFA_ERR_INVALID_ARG;  // an empty lse may have no storage
   if ((st = check_mask(mask)) != MFA_OK) return st;
-  if (!mask->map) return MFA_ERR_INVALID_ARG;
-  const mfa_tile_map* map = mask->map;
-  if ((st = check_map_matches(mask, map)) != MFA_OK) return st;
-  if (map->kind != mask->kind) return MFA_ERR_SHAPE_MISMATCH;
   if (q->dtype != k->dtype || q->dtype != v->dtype || out->dtype != q->dtype) return MFA_ERR_INVALID_ARG;
   if (k->B != q->B || v->B != q->B || out->B != q->B) return MFA_ERR_SHAPE_MISMATCH;
   if (k->H != v->H || k->N != v->N || k->D != q->D || v->D != q->D) return MFA_ERR_SHAPE_MISMATCH;
@@ -942,13 +938,26 @@ mfa_status fwd_impl(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* 
   if (mask->Hm != 1 && mask->Hm != q->H) return MFA_ERR_SHAPE_MISMATCH;
   if (q->D != 64 && q->D != 128) return MFA_ERR_UNSUPPORTED;
   if (q->N > (int64_t(1) << 30) || k->N > (int64_t(1) << 30) || q->H > 65535) return MFA_ERR_UNSUPPORTED;
-  if (q->dtype == MFA_F32) {
-    if (bias_kind != MFA_BIAS_NONE) return MFA_ERR_UNSUPPORTED;  // the fp32 path takes no bias
-    return launch_fwd_f32(q, k, v, mask, map, out, lse, static_cast<cudaStream_t>(stream));
-  }
+  if (q->dtype == MFA_F32) return bias_kind != MFA_BIAS_NONE ? MFA_ERR_UNSUPPORTED : MFA_OK;  // no fp32 bias
+  const int64_t G = q->H / k->H;
+  if (block_q == 64 && (mask->Hm != 1 || G % 2 != 0)) return MFA_ERR_UNSUPPORTED;  // two heads per 64-row tile
+  return MFA_OK;
+}
+
+namespace {
+mfa_status fwd_impl(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v, const mfa_mask_desc* mask,
+                    const mfa_bias* bias, const mfa_tensor* out, float* lse, void* stream) {
+  mfa_status st;
+  const int32_t bias_kind = bias ? bias->kind : MFA_BIAS_NONE;
+  if ((st = check_mask(mask)) != MFA_OK) return st;
+  if (!mask->map) return MFA_ERR_INVALID_ARG;
+  const mfa_tile_map* map = mask->map;
+  if ((st = check_map_matches(mask, map)) != MFA_OK) return st;
+  if (map->kind != mask->kind) return MFA_ERR_SHAPE_MISMATCH;
+  if ((st = check_fwd_args(q, k, v, mask, bias, out, lse, map->block_q)) != MFA_OK) return st;
+  if (q->dtype == MFA_F32) return launch_fwd_f32(q, k, v, mask, map, out, lse, static_cast<cudaStream_t>(stream));
   const int G = static_cast<int>(q->H / k->H);
   const int GP = map->block_q == 64 ? 2 : 1;
-  if (GP == 2 && (mask->Hm != 1 || G % 2 != 0)) return MFA_ERR_UNSUPPORTED;
   if (q->N == 0) return MFA_OK;
 
   FwdParams p;

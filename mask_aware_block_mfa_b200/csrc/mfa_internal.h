@@ -133,6 +133,12 @@ inline mfa_status check_map_matches(const mfa_mask_desc* d, const mfa_tile_map* 
   return MFA_OK;
 }
 
+// Every host-side check mfa_fwd / mfa_fwd_bias make on their arguments except
+// those on the tile map itself, for a map with `block_q`-row tiles (bias may
+// be NULL). MFA_OK when the forward pass can run.
+mfa_status check_fwd_args(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v, const mfa_mask_desc* mask,
+                          const mfa_bias* bias, const mfa_tensor* out, const float* lse, int32_t block_q);
+
 // fp32 inputs: the same tile map walked by an fp32 CUDA-core kernel
 // (fwd_f32_simt.cu). Arguments are already validated by mfa_fwd.
 mfa_status launch_fwd_f32(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v, const mfa_mask_desc* mask,

@@ -12,8 +12,11 @@
 // The array is a file-scope __device__ variable of MFA_NOALLOC_SCRATCH_BYTES.
 // Every GPU on which the library's kernels are loaded holds one copy until the
 // process exits. Host code cannot use the variable's name as a device address,
-// so the first call on each device looks the address up with
-// cudaGetSymbolAddress (with that device current) and caches it per device.
+// so the address is looked up with cudaGetSymbolAddress, with the call's device
+// current: on the first call on each device, and again on every later call
+// made while the stream is not capturing (after a cudaDeviceReset the module is
+// loaded anew and the array may sit elsewhere). A call on a capturing stream
+// uses the address the last lookup on that device found.
 // All calls on a device share the one array: calls that overlap on the GPU
 // race with each other and must be ordered by the caller (one stream, or
 // events between streams).
@@ -35,13 +38,15 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[MFA_NOALLOC_SCRATCH_BY
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of this device's copy of the scratch array (set up on the
-// first call per device; nullptr if the lookup fails).
-void* device_scratch() {
+// Device address of the current device's copy of the scratch array (nullptr
+// if the lookup fails or no address is known while `stream` is capturing).
+void* device_scratch(cudaStream_t stream) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return nullptr;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone || !g_scratch_addr[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return nullptr;
     g_scratch_addr[dev] = ptr;
@@ -61,7 +66,10 @@ extern "C" mfa_status mfa_fwd_noalloc(const mfa_tensor* q, const mfa_tensor* k, 
   const size_t need = mfa_tile_map_bytes(mask->B, mask->Hm, mask->Nq, mask->Nk, block_q, block_k);
   if (need == 0) return MFA_ERR_UNSUPPORTED;                    // block sizes other than 64 / 128
   if (need > MFA_NOALLOC_SCRATCH_BYTES) return MFA_ERR_UNSUPPORTED;  // the map does not fit the array
-  void* buf = device_scratch();
+  // Everything mfa_fwd would reject is rejected here, before the map build
+  // launches anything or touches the shared array.
+  if ((st = check_fwd_args(q, k, v, mask, nullptr, out, lse, block_q)) != MFA_OK) return st;
+  void* buf = device_scratch(static_cast<cudaStream_t>(stream));
   if (!buf) return MFA_ERR_CUDA;
   mfa_tile_map map;
   st = mfa_tile_map_init(&map, buf, MFA_NOALLOC_SCRATCH_BYTES, mask->B, mask->Hm, mask->Nq, mask->Nk, block_q,

@@ -339,3 +339,46 @@ def test_mask_and_map_arrays_must_share_the_call_device():
     B._same_device(q, same)
     with pytest.raises(ValueError, match="mask or tile-map array"):
         B._same_device(q, same, other)
+
+
+def _noalloc(lib, q, k, v, d, o, bq=64, bk=128, lse=0x7200_0000_0000):
+    return lib.mfa_fwd_noalloc(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.byref(d), bq, bk,
+                               ctypes.byref(o), lse, None, None)
+
+
+def test_noalloc_rejects_what_fwd_rejects_before_any_launch(lib):
+    """mfa_fwd_noalloc runs mfa_fwd's host checks before its map build: every
+    call below returns without a CUDA call (this machine has no GPU, so a call
+    that reached the device would fail with MFA_ERR_CUDA instead)."""
+    m = _fake_map(lib)
+    d = _fake_mask(m)
+    q, k, v, o = _fake_tensor(1, 8, 512, 128), _fake_tensor(1, 2, 512, 128), _fake_tensor(1, 2, 512, 128), \
+        _fake_tensor(1, 8, 512, 128)
+    assert _noalloc(lib, q, k, v, d, o, lse=0) == B.MFA_ERR_INVALID_ARG
+    assert _noalloc(lib, _fake_tensor(1, 8, 512, 128, addr=0), k, v, d, o) == B.MFA_ERR_INVALID_ARG
+    assert _noalloc(lib, _fake_tensor(1, 8, 512, 128, dtype=B.MFA_F32), k, v, d, o) == B.MFA_ERR_INVALID_ARG
+    assert _noalloc(lib, _fake_tensor(1, 8, 512, 96), _fake_tensor(1, 2, 512, 96), _fake_tensor(1, 2, 512, 96), d,
+                    _fake_tensor(1, 8, 512, 96)) == B.MFA_ERR_UNSUPPORTED
+    assert _noalloc(lib, q, _fake_tensor(1, 3, 512, 128), _fake_tensor(1, 3, 512, 128), d, o) == \
+        B.MFA_ERR_SHAPE_MISMATCH
+    assert _noalloc(lib, q, k, v, d, _fake_tensor(1, 8, 256, 128)) == B.MFA_ERR_SHAPE_MISMATCH
+    unaligned = _fake_tensor(1, 8, 512, 128, addr=0x7100_0000_0002)
+    assert _noalloc(lib, unaligned, k, v, d, o) == B.MFA_ERR_UNSUPPORTED
+    # two heads per 64-row tile need an even group size
+    q6, o6 = _fake_tensor(1, 6, 512, 128), _fake_tensor(1, 6, 512, 128)
+    assert _noalloc(lib, q6, k, v, d, o6) == B.MFA_ERR_UNSUPPORTED
+    assert _noalloc(lib, q, k, v, d, o, bq=96) == B.MFA_ERR_UNSUPPORTED
+    assert _noalloc(lib, q, k, v, _fake_mask(m, Nq=256), o) == B.MFA_ERR_SHAPE_MISMATCH
+
+
+def test_binding_rejects_a_stream_of_another_device():
+    """The binding launches on the tensors' device; a stream of another device is refused."""
+    import torch
+
+    class FakeStream:
+        device = torch.device("cuda", 1)
+        cuda_stream = 0
+
+    with pytest.raises(ValueError, match="stream is on"):
+        B._stream_ptr(FakeStream(), torch.device("cuda", 0))
+    assert B._stream_ptr(FakeStream(), torch.device("cuda", 1)) == 0

@@ -67,3 +67,42 @@ def test_noalloc_rejects_maps_beyond_its_array():
     fake = B.MfaTensor()
     code = lib.mfa_fwd_noalloc(fake, fake, fake, desc, 64, 64, fake, None, None, None)
     assert code == B.MFA_ERR_UNSUPPORTED
+
+
+def test_noalloc_matches_the_oracle():
+    """One case checked against the float64 CPU oracle directly, so this file
+    stands on its own and does not rely only on the regular path's parity."""
+    from oracle import attention as OA
+    mask = W.make_mask("doc8k", N=1536)
+    q, k, v = _problem(mask, 4, 2, 128, seed=37)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    B.fwd_noalloc(q, k, v, B.DeviceMask(mask), 64, 128, out, lse)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = OA.attention(q.cpu(), k.cpu(), v.cpu(), mask)
+    compare_attention(out.float().cpu(), lse.cpu(), ref_out, ref_lse)
+
+
+def test_noalloc_reports_device_errors_through_dev_err():
+    """A column bound outside [0, Nq] is found by the map build on the device
+    (MFA_DEVERR_BOUNDS, no fault); the bits reach the caller's dev_err. The
+    next call with a valid mask clears them, and a call with dev_err = None
+    skips the copy and still computes."""
+    mask = W.make_mask("tiny_doc_fp32", N=256)
+    bad = W.MaskDesc(**{**mask.__dict__})
+    bad.lte = mask.lte.copy()
+    bad.lte[0, 0, 5] = 256 + 7
+    q, k, v = _problem(mask, 4, 2, 128, seed=41)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    dev_err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    B.fwd_noalloc(q, k, v, B.DeviceMask(bad), 64, 64, out, lse, dev_err)
+    torch.cuda.synchronize()
+    assert int(dev_err.item()) & B.DEVERR_BOUNDS
+    B.fwd_noalloc(q, k, v, B.DeviceMask(mask), 64, 64, out, lse, dev_err)
+    torch.cuda.synchronize()
+    assert int(dev_err.item()) == 0
+    out2 = torch.full_like(q, float("nan"))
+    B.fwd_noalloc(q, k, v, B.DeviceMask(mask), 64, 64, out2, lse, None)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, out)
