@@ -303,6 +303,18 @@ mfa_status mfa_fwd_noalloc(const mfa_tensor* q, const mfa_tensor* k, const mfa_t
                            const mfa_mask_desc* mask, int32_t block_q, int32_t block_k,
                            const mfa_tensor* out, float* lse, uint32_t* dev_err, void* stream);
 
+/* Test hook for the bounded waits of the forward kernel; the pages have no
+ * counterpart. Every wait of the bf16 forward pipeline gives up after a time
+ * limit (2 s by default): the CTA then unwinds (its roles leave, copies already
+ * issued land, TMEM is released), MFA_DEVERR_TIMEOUT is set in the map's error
+ * word and that launch's outputs are invalid. Arming this hook makes the next
+ * bf16 mfa_fwd / mfa_fwd_bias launch in the process use a limit of wait_us
+ * microseconds and have CTA 0 withhold its first K tile (it issues no copy and
+ * no arrival for it), so that one wait runs out; the hook then disarms itself.
+ * Nothing faults: the wait that runs out is on a tile no copy will ever fill.
+ * wait_us in [1, 1000000], else MFA_ERR_INVALID_ARG. Host only. */
+mfa_status mfa_test_arm_fwd_timeout(uint32_t wait_us);
+
 /* Bytes of the DEVICE workspace mfa_bwd needs for these shapes (0 on invalid
  * shapes). Host only. */
 size_t mfa_bwd_workspace_bytes(int32_t B, int32_t Hq, int32_t Nq, int32_t Nk, int32_t D);

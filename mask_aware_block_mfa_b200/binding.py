@@ -25,7 +25,7 @@ DEVERR_BOUNDS, DEVERR_SEL, DEVERR_TIMEOUT, DEVERR_MAP = 1, 2, 4, 8
 EXPORTS = ("mfa_abi_version", "mfa_status_string", "mfa_tile_map_bytes", "mfa_tile_map_init",
            "mfa_build_tile_map", "mfa_fwd", "mfa_fwd_noalloc", "mfa_get_device_status",
            "mfa_mask_from_sparse_mode", "mfa_bwd_workspace_bytes", "mfa_bwd", "mfa_decode_workspace_bytes",
-           "mfa_decode", "mfa_fwd_bias")
+           "mfa_decode", "mfa_fwd_bias", "mfa_test_arm_fwd_timeout")
 BIAS_NONE, BIAS_ALIBI, BIAS_ALIBI_SQRT, BIAS_ALIBI_LEFT = 0, 1, 2, 3
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -121,6 +121,8 @@ def load(path: str = _LIB_PATH) -> ctypes.CDLL:
                                                                  ctypes.POINTER(MfaTensor), ctypes.c_void_p,
                                                                  ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
                                                                  ctypes.c_void_p, ctypes.c_void_p]
+    lib.mfa_test_arm_fwd_timeout.restype = ctypes.c_int
+    lib.mfa_test_arm_fwd_timeout.argtypes = [ctypes.c_uint32]
     if lib.mfa_abi_version() != 1:
         raise RuntimeError("libmfa.so ABI version mismatch")
     _lib = lib
@@ -424,6 +426,13 @@ class Decode:
         """Synchronise and return the device error bits (0 = none)."""
         torch.cuda.synchronize()
         return 0 if self.err is None else int(self.err.item())
+
+
+def arm_fwd_timeout_test(wait_us: int) -> None:
+    """Test hook: the next bf16 forward launch withholds one K tile and uses a
+    wait limit of wait_us microseconds, so one bounded wait runs out (see
+    mfa_test_arm_fwd_timeout in mfa.h)."""
+    _check("mfa_test_arm_fwd_timeout", load().mfa_test_arm_fwd_timeout(int(wait_us)))
 
 
 def device_status(tmap: TileMap, stream=None) -> int:

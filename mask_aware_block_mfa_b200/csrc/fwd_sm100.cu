@@ -74,12 +74,13 @@ struct FwdParams {
   const int32_t* order;
   __nv_bfloat16* out;
   int64_t os0, os1, os2;
-  int32_t out_v8;  // 1: out and its strides are 32-byte aligned (256-bit stores)
   float* lse;
   uint32_t* err;
   uint32_t* sched;  // [0] next work item, [1] CTAs finished (map scratch words)
   int32_t bias_kind;     // MFA_BIAS_* (kernels instantiated with kBias only)
   const float* slopes;   // [Hq] ALiBi slopes
+  uint64_t wait_ns;      // limit of every bounded wait on the pipeline (kWaitTimeoutNs)
+  int32_t withhold_k;    // test hook: 1 = CTA 0 never loads its first K tile (see mfa_test_arm_fwd_timeout)
 };
 
 constexpr int kRing = 4;  // decoded work items in flight from the producer to the other roles
@@ -93,7 +94,11 @@ struct Cfg {
   static constexpr int kQ = 0;  // two Q slots
   static constexpr int kK = kQ + 2 * kQBytes;
   static constexpr int kV = kK + kStages * kKVBytes;
-  static constexpr int kBar = kV + kStages * kKVBytes;
+  // Output staging for the TMA-store epilogue: one 32-row x 32-column bf16
+  // tile (2 KB, 64-byte swizzle) per softmax warp.
+  static constexpr int kStage = kV + kStages * kKVBytes;
+  static constexpr int kStageBytes = 32 * 32 * 2;
+  static constexpr int kBar = kStage + 8 * kStageBytes;
   // q_full[2] q_empty[2] k_full[S] k_empty[S] v_full[S] v_empty[S] s_full[2] p_full[2]
   // s_full[2][2] p_full[2][2] o_done[2] pv_done[2] bnd[2][2] drain sched_full[kRing] sched_empty[kRing]
   static constexpr int kNumBars = 4 + 4 * kStages + 12 + 4 + 1 + 2 * kRing;
@@ -229,7 +234,8 @@ __device__ __forceinline__ uint32_t transpose32_warp(uint32_t x, int lane) {
 template <int D, int BK, int GP, int kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     mfa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                   const FwdParams p) {
   using C = Cfg<D, BK>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -257,7 +263,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   WorkItem* ring = reinterpret_cast<WorkItem*>(smem + C::kRingOff);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
-  uint32_t* s_epi = reinterpret_cast<uint32_t*>(smem + C::kMisc + 8);  // tile 0's finished epilogue warps
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wg = warp >> 2;
@@ -288,11 +293,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sched_empty[i], 1 + 8);  // the MMA thread and one lane of each softmax warp
     }
     *s_abort = 0;
-    *s_epi = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, C::kTmemCols);
@@ -316,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the next one. The producer decodes it once and publishes it.
       for (int it = 0; !stop; ++it) {
         const int rs = it % kRing;
-        if (it >= kRing && !mbar_wait(&sched_empty[rs], ((it / kRing) - 1) & 1, s_abort)) break;
+        if (it >= kRing && !mbar_wait(&sched_empty[rs], ((it / kRing) - 1) & 1, s_abort, p.wait_ns)) break;
         const uint32_t wu = atomicAdd(&p.sched[0], 1u);
         WorkItem info;
         info.w = wu < static_cast<uint32_t>(p.n_items) ? static_cast<int>(wu) : -1;
@@ -329,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hkv = info.hkv;
         for (int s = 0; s < 2 && !stop; ++s) {
           if (t[s].n == 0) continue;
-          if (quse[s] > 0 && !mbar_wait(&q_empty[s], (quse[s] - 1) & 1, s_abort)) { stop = true; break; }
+          if (quse[s] > 0 && !mbar_wait(&q_empty[s], (quse[s] - 1) & 1, s_abort, p.wait_ns)) { stop = true; break; }
           mbar_arrive_expect_tx(&q_full[s], C::kQBytes);
           uint8_t* dst = sQ + s * C::kQBytes;
 #pragma unroll
@@ -354,13 +359,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int st = kv_it % S;
           const uint32_t ph = (kv_it / S) & 1;
-          if (kv_it >= S && !mbar_wait(&k_empty[st], ph ^ 1, s_abort)) { stop = true; break; }
-          mbar_arrive_expect_tx(&k_full[st], C::kKVBytes);
+          if (kv_it >= S && !mbar_wait(&k_empty[st], ph ^ 1, s_abort, p.wait_ns)) { stop = true; break; }
+          // Test hook: the first K tile of CTA 0 is neither loaded nor
+          // announced, so the MMA warp's bounded wait for it runs out.
+          const bool withhold = p.withhold_k && blockIdx.x == 0 && kv_it == 0;
+          if (!withhold) {
+            mbar_arrive_expect_tx(&k_full[st], C::kKVBytes);
 #pragma unroll
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_4d(sK + st * C::kKVBytes + c * (BK * 128), &tm_k, &k_full[st], c * 64, kt * BK, hkv, t[0].b);
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_4d(sK + st * C::kKVBytes + c * (BK * 128), &tm_k, &k_full[st], c * 64, kt * BK, hkv, t[0].b);
+          }
           k_inflight = kv_it + 1;
-          if (kv_it >= S && !mbar_wait(&v_empty[st], ph ^ 1, s_abort)) { stop = true; break; }
+          if (kv_it >= S && !mbar_wait(&v_empty[st], ph ^ 1, s_abort, p.wait_ns)) { stop = true; break; }
           mbar_arrive_expect_tx(&v_full[st], C::kKVBytes);
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c)
@@ -375,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s)
           if (quse[s] > 0) mbar_wait(&q_full[s], (quse[s] - 1) & 1, &no_abort);
         for (uint32_t j = (k_inflight > S ? k_inflight - S : 0); j < k_inflight; ++j)
-          mbar_wait(&k_full[j % S], (j / S) & 1, &no_abort);
+          if (!(p.withhold_k && blockIdx.x == 0 && j == 0)) mbar_wait(&k_full[j % S], (j / S) & 1, &no_abort);
         for (uint32_t j = (v_inflight > S ? v_inflight - S : 0); j < v_inflight; ++j)
           mbar_wait(&v_full[j % S], (j / S) & 1, &no_abort);
       }
@@ -410,9 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O_t += P_t V for the tile's pending k-tile.
       auto issue_pv = [&](int s) -> bool {
         const uint32_t sb = psq[s] % C::kSBufs;
-        if (!warp_all(mbar_wait(&p_full[2 * s + sb], (psq[s] / C::kSBufs) & 1, s_abort))) return false;
+        if (!warp_all(mbar_wait(&p_full[2 * s + sb], (psq[s] / C::kSBufs) & 1, s_abort, p.wait_ns))) return false;
         const uint32_t vst = pkv[s] % S;
-        if (!warp_all(mbar_wait(&v_full[vst], (pkv[s] / S) & 1, s_abort))) return false;
+        if (!warp_all(mbar_wait(&v_full[vst], (pkv[s] / S) & 1, s_abort, p.wait_ns))) return false;
         tc_fence_after();
         const uint32_t a_p = tmem + (s * C::kSBufs + sb) * BK;
         const uint32_t d_o = tmem + C::kOCol + s * D;
@@ -436,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       for (int it = 0; ok; ++it) {
         const int rs = it % kRing;
-        if (!(ok = warp_all(mbar_wait(&sched_full[rs], (it / kRing) & 1, s_abort)))) break;
+        if (!(ok = warp_all(mbar_wait(&sched_full[rs], (it / kRing) & 1, s_abort, p.wait_ns)))) break;
         const WorkItem info = ring[rs];
         if (lane == 0) mbar_arrive(&sched_empty[rs]);
         if (info.w < 0) break;
@@ -461,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if ((pv & 1u) && !(ok = issue_pv(0))) break;
             if ((pv & 2u) && !warp_all(mbar_try_wait(&k_full[st], ph)) && !(ok = issue_pv(1))) break;
           }
-          if (!(ok = warp_all(mbar_wait(&k_full[st], ph, s_abort)))) break;
+          if (!(ok = warp_all(mbar_wait(&k_full[st], ph, s_abort, p.wait_ns)))) break;
           tc_fence_after();
           // S_s = Q_s K^T for k-tile st; returns the pending-P.V flags it adds.
           auto issue_s = [&](int s) -> uint32_t {
@@ -485,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           };
           auto q_ready = [&](int s) -> bool {
             if (qready[s]) return true;
-            if (!warp_all(mbar_wait(&q_full[s], quse[s] & 1, s_abort))) return false;
+            if (!warp_all(mbar_wait(&q_full[s], quse[s] & 1, s_abort, p.wait_ns))) return false;
             tc_fence_after();
             qready[s] = true;
             return true;
@@ -561,12 +571,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool k_ragged = (p.Nk % BK) != 0;
     int4* my_bounds = s_bounds + slot * 2 * BK;
     uint64_t* my_bnd = bnd_full + 2 * slot;
-    uint32_t s_cnt = 0, o_cnt = 0, n_bnd = 0, epi_items = 0;
+    uint32_t s_cnt = 0, o_cnt = 0, n_bnd = 0;
     bool ok = true;
 
     for (int it = 0; ok; ++it) {
       const int rs = it % kRing;
-      if (!(ok = warp_all(mbar_wait(&sched_full[rs], (it / kRing) & 1, s_abort)))) break;
+      if (!(ok = warp_all(mbar_wait(&sched_full[rs], (it / kRing) & 1, s_abort, p.wait_ns)))) break;
       const WorkItem info = ring[rs];
       __syncwarp();
       if (lane == 0) mbar_arrive(&sched_empty[rs]);
@@ -609,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[r] = v;
           }
           mbar_arrive(&my_bnd[bs]);
-          if (!(ok = warp_all(mbar_wait(&my_bnd[bs], (n_bnd >> 1) & 1, s_abort)))) break;
+          if (!(ok = warp_all(mbar_wait(&my_bnd[bs], (n_bnd >> 1) & 1, s_abort, p.wait_ns)))) break;
           bnd = dst;
           ++n_bnd;
         }
@@ -657,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // S number s_cnt of this tile sits in buffer s_cnt % kSBufs.
         const uint32_t sb = s_cnt % C::kSBufs;
         const uint32_t tmem_s = tmem + (slot * C::kSBufs + sb) * BK;
-        if (!(ok = warp_all(mbar_wait(&s_full[2 * slot + sb], (s_cnt / C::kSBufs) & 1, s_abort)))) break;
+        if (!(ok = warp_all(mbar_wait(&s_full[2 * slot + sb], (s_cnt / C::kSBufs) & 1, s_abort, p.wait_ns)))) break;
         ++s_cnt;
         tc_fence_after();
 
@@ -736,7 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // S buffers, S number k is issued before the P.V of S number k - 1,
           // so that P.V (phase k - 1 of pv_done; at most one phase is pending)
           // must complete before O is rescaled.
-          if (C::kSBufs == 2 && !(ok = warp_all(mbar_wait(&pv_done[slot], (s_cnt - 2) & 1, s_abort)))) break;
+          if (C::kSBufs == 2 && !(ok = warp_all(mbar_wait(&pv_done[slot], (s_cnt - 2) & 1, s_abort, p.wait_ns)))) break;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -758,58 +768,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The next item's first P.V into this slot's O waits for this warpgroup's
       // next P, which is written after these reads, so O needs no other guard.
       if (n > 0) {
-        if (!(ok = warp_all(mbar_wait(&o_done[slot], o_cnt & 1, s_abort)))) break;
+        if (!(ok = warp_all(mbar_wait(&o_done[slot], o_cnt & 1, s_abort, p.wait_ns)))) break;
         ++o_cnt;
         tc_fence_after();
       }
       const bool has = l_run > 0.f;
       const float inv = has ? 1.f / l_run : 0.f;
       const bool store = qi < p.Nq;
-      __nv_bfloat16* orow = p.out + static_cast<int64_t>(T.b) * p.os0 + static_cast<int64_t>(head) * p.os1 +
-                            static_cast<int64_t>(qi) * p.os2;
-      // In kind-0 items both tiles finish together and their row stores would
-      // share the load/store unit; tile 1 stores after tile 0 has issued its
-      // stores, so tile 0 goes on to its next item earlier and the tiles end up
-      // staggered. The count of tile 0's finished warps only grows, so a wait
-      // cannot confuse one item with another; the spin is bounded.
-      if (slot == 1 && p.item_kind == 0) {
-        const uint32_t want = 4u * ++epi_items;
-        uint64_t t0 = 0;
-        for (uint32_t k = 0; *reinterpret_cast<volatile uint32_t*>(s_epi) < want; ++k) {
-          if ((k & 255) == 255) {
-            if (t0 == 0) t0 = global_timer_ns();
-            if (*s_abort || global_timer_ns() - t0 > kWaitTimeoutNs) {
-              *s_abort = 1;
-              ok = false;
-              break;
-            }
-          }
-        }
-        if (!(ok = warp_all(ok))) break;
-      }
-      // Each thread writes its own row. With 32-byte aligned rows a store
-      // covers whole 32-byte sectors; 16-byte stores would write every sector
-      // in two halves from two instructions. The chunk loop stays rolled: it
-      // runs once per item.
+      // Each warp writes its 32 rows through its own staging tile, 32 columns
+      // at a time: every lane puts its row's 64 bytes into shared memory
+      // (64-byte swizzle: 16-byte unit j of row l at unit j ^ ((l >> 1) & 3),
+      // conflict-free), and one lane hands the tile to a TMA store, which clips
+      // rows past Nq. The stores leave the warp at once; a staging tile is
+      // rewritten only after the TMA has read its previous contents.
+      {
+        const int row0 = (GP == 2) ? T.q0 + ((sw * 32) & 63) : T.q0 + sw * 32;
+        const int hd = (GP == 2) ? T.h0 + (sw >> 1) : T.h0;
+        const uint32_t stg = smem_u32(smem + C::kStage + (slot * 4 + sw) * C::kStageBytes);
+        const uint32_t my_row = stg + lane * 64;
+        const uint32_t swz = (lane >> 1) & 3;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (n > 0) {
-          tmem_ld_32x32b_x32(tmem_o + lane_off + c * 32, o);
-          tmem_ld_wait();
-        }
-        if (store) {
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          if (n > 0) {
+            tmem_ld_32x32b_x32(tmem_o + lane_off + c * 32, o);
+            tmem_ld_wait();
+          }
           uint32_t w[16];
 #pragma unroll
           for (int u = 0; u < 16; ++u)
             w[u] = has ? pack_bf16x2(__uint_as_float(o[2 * u]) * inv, __uint_as_float(o[2 * u + 1]) * inv) : 0u;
-          if (p.out_v8) {
-            st_global_v8(orow + c * 32, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
-            st_global_v8(orow + c * 32 + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
-          } else {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
 #pragma unroll
-            for (int g = 0; g < 4; ++g)
-              reinterpret_cast<uint4*>(orow)[c * 4 + g] = make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+          for (int j = 0; j < 4; ++j)
+            st_shared_v4(my_row + ((j ^ swz) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_4d(&tm_o, smem + C::kStage + (slot * 4 + sw) * C::kStageBytes, c * 32, row0, hd, T.b);
+            bulk_commit_group();
           }
         }
       }
@@ -817,12 +815,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float lse = has ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
         p.lse[(static_cast<size_t>(T.b) * p.Hq + head) * p.Nq + qi] = lse;
       }
-      if (slot == 0 && p.item_kind == 0) {
-        __syncwarp();
-        if (lane == 0) atomicAdd(s_epi, 1u);
-      }
     }
     if (!ok && lane == 0) atomicOr(p.err, MFA_DEVERR_TIMEOUT);
+    // The warp's TMA stores must be complete before its staging tile and the
+    // CTA go away.
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   __syncthreads();
@@ -860,6 +858,23 @@ bool make_map(CUtensorMap* map, const mfa_tensor* t, int box_rows) {
   return r == CUDA_SUCCESS;
 }
 
+// The output as TMA-store destination: 32-column x 32-row boxes with the
+// 64-byte swizzle of the kernel's staging tiles.
+bool make_store_map(CUtensorMap* map, const mfa_tensor* t) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(t->D), static_cast<cuuint64_t>(t->N),
+                        static_cast<cuuint64_t>(t->H), static_cast<cuuint64_t>(t->B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(t->stride[2]) * 2, static_cast<cuuint64_t>(t->stride[1]) * 2,
+                           static_cast<cuuint64_t>(t->stride[0]) * 2};
+  cuuint32_t box[4] = {32, 32, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t->data, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 mfa_status check_tensor(const mfa_tensor* t) {
   if (!t) return MFA_ERR_INVALID_ARG;
   if (t->B <= 0 || t->H <= 0 || t->N < 0 || t->D <= 0) return MFA_ERR_INVALID_ARG;
@@ -873,8 +888,8 @@ mfa_status check_tensor(const mfa_tensor* t) {
 }
 
 template <int D, int BK, int GP, int kBias>
-mfa_status launch_b(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
-                    cudaStream_t s) {
+mfa_status launch_b(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                    const FwdParams& p, cudaStream_t s) {
   using C = Cfg<D, BK>;
   static std::atomic<uint64_t> attr_devs{0};
   if (!ensure_smem_attr(reinterpret_cast<const void*>(mfa_fwd_kernel<D, BK, GP, kBias>), C::kAlloc, attr_devs))
@@ -882,16 +897,16 @@ mfa_status launch_b(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
   const int sms = device_sm_count();
   if (sms <= 0) return MFA_ERR_CUDA;
   const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: at most one CTA per SM
-  mfa_fwd_kernel<D, BK, GP, kBias><<<grid, kThreads, C::kAlloc, s>>>(mq, mk, mv, p);
+  mfa_fwd_kernel<D, BK, GP, kBias><<<grid, kThreads, C::kAlloc, s>>>(mq, mk, mv, mo, p);
   return cudaGetLastError() == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
 }
 
 template <int D, int BK, int GP>
-mfa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
-                  cudaStream_t s) {
-  if (p.bias_kind == MFA_BIAS_NONE) return launch_b<D, BK, GP, 0>(mq, mk, mv, p, s);
-  if (p.bias_kind == MFA_BIAS_ALIBI_SQRT) return launch_b<D, BK, GP, 2>(mq, mk, mv, p, s);
-  return launch_b<D, BK, GP, 1>(mq, mk, mv, p, s);
+mfa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                  const FwdParams& p, cudaStream_t s) {
+  if (p.bias_kind == MFA_BIAS_NONE) return launch_b<D, BK, GP, 0>(mq, mk, mv, mo, p, s);
+  if (p.bias_kind == MFA_BIAS_ALIBI_SQRT) return launch_b<D, BK, GP, 2>(mq, mk, mv, mo, p, s);
+  return launch_b<D, BK, GP, 1>(mq, mk, mv, mo, p, s);
 }
 
 }  // namespace
@@ -899,6 +914,9 @@ mfa_status launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMa
 
 namespace mfa {
 namespace {
+// Armed by mfa_test_arm_fwd_timeout: the wait limit in microseconds for the
+// next bf16 forward launch, which then withholds one K tile (0 = not armed).
+std::atomic<uint32_t> g_timeout_test_us{0};
 mfa_status fwd_impl(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v, const mfa_mask_desc* mask,
                     const mfa_bias* bias, const mfa_tensor* out, float* lse, void* stream);
 }  // namespace
@@ -907,6 +925,12 @@ mfa_status fwd_impl(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* 
 extern "C" mfa_status mfa_fwd(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v,
                               const mfa_mask_desc* mask, const mfa_tensor* out, float* lse, void* stream) {
   return mfa::fwd_impl(q, k, v, mask, nullptr, out, lse, stream);
+}
+
+extern "C" mfa_status mfa_test_arm_fwd_timeout(uint32_t wait_us) {
+  if (wait_us == 0 || wait_us > 1000000u) return MFA_ERR_INVALID_ARG;
+  mfa::g_timeout_test_us.store(wait_us);
+  return MFA_OK;
 }
 
 extern "C" mfa_status mfa_fwd_bias(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v,
@@ -987,31 +1011,35 @@ mfa_status fwd_impl(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* 
   p.cls = map->tile_class; p.list = map->tile_list; p.count = map->tile_count; p.order = map->order;
   p.out = static_cast<__nv_bfloat16*>(out->data);
   p.os0 = out->stride[0]; p.os1 = out->stride[1]; p.os2 = out->stride[2];
-  p.out_v8 = (reinterpret_cast<uintptr_t>(out->data) % 32 == 0 && out->stride[0] % 16 == 0 &&
-              out->stride[1] % 16 == 0 && out->stride[2] % 16 == 0)
-                 ? 1
-                 : 0;
   p.lse = lse;
   p.err = map->err;
   p.sched = map->err + 1;
   p.bias_kind = bias_kind;
   p.slopes = bias_kind != MFA_BIAS_NONE ? bias->slopes : nullptr;
+  p.wait_ns = kWaitTimeoutNs;
+  p.withhold_k = 0;
+  const uint32_t armed_us = g_timeout_test_us.exchange(0u);
+  if (armed_us != 0) {
+    p.wait_ns = static_cast<uint64_t>(armed_us) * 1000u;
+    p.withhold_k = 1;
+  }
   if (n_items64 <= 0) return MFA_OK;
   if (n_items64 > 0x7fffffff) return MFA_ERR_UNSUPPORTED;
   p.n_items = static_cast<int32_t>(n_items64);
 
   // With Nk == 0 every list is empty and the K/V maps are never read.
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   memset(&mk, 0, sizeof(mk));
   memset(&mv, 0, sizeof(mv));
   if (!make_map(&mq, q, 64)) return MFA_ERR_CUDA;
+  if (!make_store_map(&mo, out)) return MFA_ERR_CUDA;
   if (k->N > 0 && (!make_map(&mk, k, map->block_k) || !make_map(&mv, v, map->block_k))) return MFA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int D = static_cast<int>(q->D), BK = map->block_k;
-  if (D == 128 && BK == 128) return GP == 2 ? launch<128, 128, 2>(mq, mk, mv, p, s) : launch<128, 128, 1>(mq, mk, mv, p, s);
-  if (D == 128 && BK == 64) return GP == 2 ? launch<128, 64, 2>(mq, mk, mv, p, s) : launch<128, 64, 1>(mq, mk, mv, p, s);
-  if (D == 64 && BK == 128) return GP == 2 ? launch<64, 128, 2>(mq, mk, mv, p, s) : launch<64, 128, 1>(mq, mk, mv, p, s);
-  return GP == 2 ? launch<64, 64, 2>(mq, mk, mv, p, s) : launch<64, 64, 1>(mq, mk, mv, p, s);
+  if (D == 128 && BK == 128) return GP == 2 ? launch<128, 128, 2>(mq, mk, mv, mo, p, s) : launch<128, 128, 1>(mq, mk, mv, mo, p, s);
+  if (D == 128 && BK == 64) return GP == 2 ? launch<128, 64, 2>(mq, mk, mv, mo, p, s) : launch<128, 64, 1>(mq, mk, mv, mo, p, s);
+  if (D == 64 && BK == 128) return GP == 2 ? launch<64, 128, 2>(mq, mk, mv, mo, p, s) : launch<64, 128, 1>(mq, mk, mv, mo, p, s);
+  return GP == 2 ? launch<64, 64, 2>(mq, mk, mv, mo, p, s) : launch<64, 64, 1>(mq, mk, mv, mo, p, s);
 }
 
 }  // namespace

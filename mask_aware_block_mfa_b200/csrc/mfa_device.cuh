@@ -57,48 +57,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for a packed pair on the FMA/ALU pipes instead of the MUFU unit.
-// Cody and Waite's range reduction: x = j + f with j = round(x) (adding
-// 1.5 * 2^23 leaves round(x) in the low mantissa bits) and f in [-1/2, 1/2];
-// 2^f from the degree-3 polynomial of minimum relative error on [-1/2, 1/2]
-// (Remez exchange, coefficients from csrc/exp2_poly_fit.py, max relative error
-// 7.5e-5 in float32); 2^j is added to the exponent field. Inputs below -125
-// (masked scores are -inf) are clamped there and give about 2^-125, not 0:
-// the caller must treat a row with no visible key separately.
-constexpr float kExp2C0 = 0x1.fff692p-1f;
-constexpr float kExp2C1 = 0x1.62f31ap-1f;
-constexpr float kExp2C2 = 0x1.f0de1ap-3f;
-constexpr float kExp2C3 = 0x1.c3f76p-5f;
-
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
-  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t t = f2_add(xc, f2_pack(kShift, kShift));
-  const uint64_t j = f2_add(t, f2_pack(-kShift, -kShift));
-  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), xc);
-  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
-  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
-                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
-}
-
-// The same 2^x for one value with the coefficients as instruction immediates
-// (no registers held across a loop); same clamp at -125.
-__device__ __forceinline__ float exp2_poly1(float x) {
-  const float xc = fmaxf(x, -125.f);
-  const float t = __fadd_rn(xc, 12582912.f);
-  const float j = __fadd_rn(t, -12582912.f);
-  const float f = __fsub_rn(xc, j);
-  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   // cvt.rn.bf16x2.f32 d, a, b puts a in the upper and b in the lower half.
@@ -146,7 +104,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // caller unwinds. A correct pipeline never gets there.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t timeout_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
@@ -154,7 +113,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > timeout_ns) {
       *abort = 1;
       return false;
     }
@@ -184,6 +143,27 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m
       :: "r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)),
          "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Shared -> global tile store by TMA, tracked by the issuing thread's bulk
+// async-groups. The staging tile must be written through the generic proxy and
+// made visible to the async proxy (fence_proxy_async_smem) before the store.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* smem_src, int32_t c0, int32_t c1,
+                                             int32_t c2, int32_t c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+               :: "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk store of this thread has read its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until every committed bulk store of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 // ------------------------------------------------------------------------

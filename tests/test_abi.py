@@ -382,3 +382,8 @@ def test_binding_rejects_a_stream_of_another_device():
     with pytest.raises(ValueError, match="stream is on"):
         B._stream_ptr(FakeStream(), torch.device("cuda", 0))
     assert B._stream_ptr(FakeStream(), torch.device("cuda", 1)) == 0
+
+
+def test_timeout_hook_rejects_limits_out_of_range(lib):
+    assert lib.mfa_test_arm_fwd_timeout(0) == B.MFA_ERR_INVALID_ARG
+    assert lib.mfa_test_arm_fwd_timeout(1_000_001) == B.MFA_ERR_INVALID_ARG
