@@ -54,13 +54,12 @@ TARGET_WORKLOADS = ("doc8k", "doc32k")
 # the forward kernel on that workload (the summaries under profiles/ give the
 # command). Each entry holds the digest of the kernel sources it was taken
 # on; a changed kernel reports traffic as null until it is captured again.
-# The digests below are those of the captured sources after a host-only
-# change (shared tensor-map lookup, per-device shared-memory attribute): the
-# device code and the launch configuration are the ones captured.
 KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/fwd_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh")
 NCU_TRAFFIC = {
-    "doc8k": (135_804_672, "19480ffac4ada9d1"),
-    "doc32k": (1_031_209_472, "19480ffac4ada9d1"),
+    "doc8k": (134_846_208, "4215f15e496d475a"),
+    "shared_question8k": (135_123_456, "4215f15e496d475a"),
+    "band16k": (520_584_192, "4215f15e496d475a"),
+    "blocksel32k": (1_125_267_456, "4215f15e496d475a"),
 }
 # The same for the gradient kernel (mfa_bwd_kernel) of the backward pass.
 BWD_KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/bwd_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh",
