@@ -143,9 +143,9 @@ def test_fwd_output_layouts(layout):
 def test_fwd_rows_without_keys_inside_visible_tiles():
     """Causal mask in which queries 100..109 see no key at all while the other
     rows of their tiles do. Those rows run through PARTIAL and FULL tiles with a
-    running max of -inf; they must still give out = 0 and lse = -inf (their
-    exponentials from the FMA-pipe exp2 are about 2^-125, not 0, so the kernel
-    has to zero their row sum), and the rows around them must be unaffected."""
+    running max of -inf (every score of the row is -inf, so each exponential is
+    taken against a reference of 0); they must still give out = 0 and
+    lse = -inf, and the rows around them must be unaffected."""
     N = 600
     j = np.arange(N, dtype=np.int32)
     uts = np.zeros((1, 1, N), np.int32)
