@@ -6,33 +6,13 @@
 // once, and the list is shared by the G query heads of head g. Query row i
 // sits at position i + Nk - Nq and sees only keys at or before it (the forward
 // pass's block-selection rule when Nq == Nk). The work is a gather of whole
-// 64-key K/V blocks, so it is bound by HBM, not by the tensor cores: with G
-// query rows per block there is little to multiply, and the CUDA cores keep up
-// with the memory (for D = 256, G = 4 a 64 KB block takes ~2,850 cycles of an
-// SM's share of HBM and ~1,000 FMA cycles).
+// 64-key K/V blocks and is bound by HBM; the two products run on the tensor
+// cores, so that the CUDA cores only run the softmax of G rows.
 //
 // Split-K, as in the pull request: a list is cut into n_split parts handled by
 // different CTAs; each writes an unnormalised partial (m, l, o), and a second
 // kernel combines them. An empty part writes m = -FLT_MAX, not -inf, so the
 // combination never evaluates exp(-inf - -inf).
-//
-// CTA = (part, query row, batch x key/value head), 256 threads (8 warps).
-//   1. The list is deduplicated in shared memory (first occurrence kept,
-//      entries outside [-1, ceil(Nk / 64)) flagged, blocks after the row's
-//      position dropped) and the part's share of it taken.
-//   2. K and V blocks arrive by TMA (64-column SW128 boxes) in a two-stage ring.
-//   3. Scores: lane l holds head dimensions [DL l, DL l + DL) of all G query
-//      rows in registers (DL = D / 32); each warp takes 64 / warps keys of the
-//      block, reads each key row once (conflict-free through the swizzle) and
-//      reduces the G partial dot products across lanes by halving transposes
-//      (G - 1 + 5 - log2 G shuffles).
-//   4. Online softmax per warp: each warp keeps its own running max and sum
-//      of every query row and its own partial outputs over the keys it
-//      handles (a split-K inside the CTA), so no block-wide barrier runs per
-//      block; a stage is released by one arrival per warp.
-//   5. P.V: lane l owns the same head dimensions of all G rows for the
-//      warp's keys; the warps' partials are combined once at the end, each
-//      rescaled by 2^(its max - the row's max).
 #include <cfloat>
 #include <climits>
 #include <cmath>
@@ -50,12 +30,6 @@ namespace {
 
 constexpr int kBlk = 64;       // keys per selection block
 constexpr int kCombineThreads = 256;
-// 16 warps when the query rows and outputs fit 128 registers a thread
-// (G * D <= 1024), else 8: more warps hide more of the shared-memory and
-// shuffle latency of the one CTA that fits an SM.
-template <int D, int G>
-constexpr int kWarpsFor = G * D <= 1024 ? 16 : 8;
-
 struct DecParams {
   int32_t B, Hq, Hkv, G, Nq, Nk, nblk, sel_k, n_split;
   float scale_log2;
@@ -70,144 +44,109 @@ struct DecParams {
   uint32_t* err;
 };
 
+__device__ __forceinline__ bool warp_all_dec(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+// ---------------------------------------------------------------------------
+// The decode kernel on the tensor cores.
+//
+// S = Q K^T as one tcgen05 MMA of M = 128 rows: rows 0 .. G-1 are the G query
+// heads of the row, the other rows of the A operand read whatever follows Q in
+// shared memory and their results are never used, so Q takes 16 rows (2 KB) per
+// 64-column chunk instead of 128. N = 64 keys (one block), K = D. Lane h of the
+// softmax warp holds head h's 64 scores (TMEM lane = row), keeps its own
+// online max and sum, and writes P (bf16) over its scores. O += P V as a TS
+// MMA (P from TMEM) with N = D, into an accumulator of 128 x D fp32 columns.
+// Two S buffers: S of block n + 1 is computed while the softmax works on block
+// n. K and V of a block share a stage of a three-stage (D = 256) or six-stage
+// (D = 128) TMA ring, with their own barriers: K is released when S of the
+// block is done, V when its P.V is. The MMA warp issues whichever of the next
+// S and the oldest pending P.V is ready first.
+//
+// Warps: 0 softmax and epilogue (TMEM lanes 0-31), 1 MMA issuer and TMEM owner,
+// 2 TMA producer, 3 idle. Every wait is bounded.
+// ---------------------------------------------------------------------------
 template <int D>
-struct DecCfg {
-  static constexpr int kDL = D / 32;                 // head dimensions per lane
-  static constexpr int kTile = kBlk * D * 2;         // one K (or V) block: D / 64 boxes of 64 rows x 128 B
-  static constexpr int kStages = 3;                  // K/V ring: two blocks in flight while one is used
-  static constexpr int kK = 0;                       // [kStages]
-  static constexpr int kV = kK + kStages * kTile;    // [kStages]
-  static constexpr int kS = kV + kStages * kTile;    // list scratch, then per-warp (m, l) at the end
-  static constexpr int kList = kS + 2 * 16 * kBlk * 4;  // deduplicated list [kMaxSelK]
-  static constexpr int kMisc = kList + kMaxSelK * 4; // softmax state, counters, barriers
-  static constexpr int kBytes = kMisc + 1024;
-  // The final combine of the warps' outputs reuses the K/V ring (16 warps with
-  // G * D <= 1024 or 8 warps with G * D <= 2048); the warps' (m, l) go to the
-  // space after the ring.
-  static_assert(16 * 32 * (1024 / D * kDL + 1) * 4 <= kS, "output reduction space (16 warps)");
-  static_assert(8 * 32 * (2048 / D * kDL + 1) * 4 <= kS, "output reduction space (8 warps)");
-  static_assert(2 * 16 * 16 * 4 <= kList - kS, "per-warp (m, l)");
+struct DecTc {
+  static constexpr int kStages = D == 256 ? 3 : 6;
+  static constexpr int kQChunk = 16 * 128;                  // 16 rows x 128 B per 64-column chunk
+  static constexpr int kQ = 0;                               // D / 64 chunks
+  static constexpr int kTile = kBlk * D * 2;                 // one K (or V) block
+  static constexpr int kStage0 = 8 * 1024;                   // stages start 1024-aligned after Q
+  static constexpr int kK = 0, kV = kTile;                   // inside a stage
+  static constexpr int kStageBytes = 2 * kTile;
+  static constexpr int kList = kStage0 + kStages * kStageBytes;  // raw list [kMaxSelK], then deduplicated
+  static constexpr int kMisc = kList + 2 * kMaxSelK * 4;
+  static constexpr int kBytes = kMisc + 512 + 1024;         // + slack for 1024-byte alignment
+  static constexpr int kTmemCols = 128 + D <= 256 ? 256 : 512;  // S0 [0,64) S1 [64,128) O [128, 128 + D)
+  static_assert(kBytes <= 232448, "shared memory");
+  // M = 128 reads 16 KB from each Q chunk's base: the last one must stay inside the allocation.
+  static_assert((D / 64 - 1) * kQChunk + 16 * 1024 <= kList, "Q chunk rows beyond 16 read allocated memory");
 };
 
-// Element offset of head dimensions [c0, c0 + n) of key row r in a K/V block
-// written by TMA with 64-column SW128 boxes: box c0 / 64, 16-byte chunk
-// (c0 % 64) / 8 placed at chunk ^ (r % 8). n <= 8 and within one chunk.
-__device__ __forceinline__ uint32_t sw_off(int r, int c0) {
-  const int box = c0 >> 6, ch = (c0 & 63) >> 3;
-  return static_cast<uint32_t>(box * (kBlk * 128) + r * 128 + ((ch ^ (r & 7)) << 4) + (c0 & 7) * 2);
-}
-
-// A bf16 pair widened to a packed float pair: bf16 is the upper half of a float.
-__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
-  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-}
-
-// Head dimensions [DL lane, DL lane + DL) of key row r as DL / 2 packed pairs.
-template <int DL>
-__device__ __forceinline__ void load_row2(const uint8_t* tile, int r, int lane, uint64_t (&x)[DL / 2]) {
-  const uint8_t* p = tile + sw_off(r, lane * DL);
-  if constexpr (DL == 8) {
-    const uint4 w = *reinterpret_cast<const uint4*>(p);
-    x[0] = bf2_to_f2(w.x); x[1] = bf2_to_f2(w.y); x[2] = bf2_to_f2(w.z); x[3] = bf2_to_f2(w.w);
-  } else {
-    const uint2 w = *reinterpret_cast<const uint2*>(p);
-    x[0] = bf2_to_f2(w.x); x[1] = bf2_to_f2(w.y);
-  }
-}
-
-// Sum v[0 .. G) over the 32 lanes. Afterwards lane l holds the total of
-// value index (l >> (5 - log2 G)) in v[0]: at distance 16, 8, ... each lane
-// keeps the half of its values whose index bit matches its own lane bit and
-// adds the partner's copy of that half; the remaining steps are a butterfly.
-template <int G>
-__device__ __forceinline__ float reduce_rows(float (&v)[G], int lane) {
-  int n = G, dist = 16;
-#pragma unroll
-  for (int step = 0; step < 5; ++step, dist >>= 1) {
-    if (n > 1) {
-      const int half = n >> 1;
-      const bool upper = (lane & dist) != 0;
-#pragma unroll
-      for (int x = 0; x < G / 2; ++x) {
-        if (x < half) {
-          const float send = upper ? v[x] : v[x + half];
-          const float recv = __shfl_xor_sync(0xffffffffu, send, dist);
-          v[x] = (upper ? v[x + half] : v[x]) + recv;
-        }
-      }
-      n = half;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], dist);
-    }
-  }
-  return v[0];
-}
-
-template <int G>
-__device__ __forceinline__ int row_of_lane(int lane) {
-  constexpr int lg = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
-  // value index bits were chosen at distances 16, 8, ...: the first step's
-  // bit is the most significant bit of the index
-  int idx = 0;
-#pragma unroll
-  for (int s = 0; s < lg; ++s) idx = (idx << 1) | ((lane >> (4 - s)) & 1);
-  return idx;
-}
-
-// The first lane that holds row h's total after reduce_rows: h's bits from the
-// most significant down sit at lane bits 4, 3, ... (the inverse of row_of_lane).
-template <int G>
-__device__ __forceinline__ int owner_lane(int h) {
-  constexpr int lg = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
-  int lane = 0;
-#pragma unroll
-  for (int s = 0; s < lg; ++s) lane |= ((h >> (lg - 1 - s)) & 1) << (4 - s);
-  return lane;
-}
-
 template <int D, int G>
-__global__ void __launch_bounds__(kWarpsFor<D, G> * 32, 1)
+__global__ void __launch_bounds__(128, 1)
     mfa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const DecParams p) {
-  using C = DecCfg<D>;
-  constexpr int DL = C::kDL;
-  constexpr int kWarps = kWarpsFor<D, G>;
-  constexpr int kThreads = kWarps * 32;
-  constexpr int kKeysPerWarp = kBlk / kWarps;
-  constexpr int kCk = kKeysPerWarp < 4 ? kKeysPerWarp : 4;  // keys per softmax step
-  extern __shared__ __align__(1024) uint8_t smem[];
+  using C = DecTc<D>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = blockIdx.x, i = blockIdx.y;
   const int bg = blockIdx.z, b = bg / p.Hkv, g = bg % p.Hkv;
-  const size_t row_unit = (static_cast<size_t>(bg) * p.Nq + i);
+  const size_t row_unit = static_cast<size_t>(bg) * p.Nq + i;
 
-  int* sList = reinterpret_cast<int*>(smem + C::kList);
-  int* sCnt = reinterpret_cast<int*>(smem + C::kMisc + 192);   // [kWarps] list compaction, [16] total
-  volatile int* sFlag = reinterpret_cast<volatile int*>(sCnt + 20);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kMisc + 512);  // [kStages] block landed
-  uint64_t* empty = full + C::kStages;                                   // [kStages] every warp done with it
+  int* sRaw = reinterpret_cast<int*>(smem + C::kList);
+  int* sList = sRaw + kMaxSelK;
+  int* sCnt = reinterpret_cast<int*>(smem + C::kMisc);          // [4] per-warp counts, [4] total
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sCnt + 8);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sCnt + 9);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kMisc + 64);
+  uint64_t* k_full = bars;              // [S]
+  uint64_t* k_empty = k_full + S;       // [S]: S of the block is done with K
+  uint64_t* v_full = k_empty + S;       // [S]
+  uint64_t* v_empty = v_full + S;       // [S]: P.V of the block is done with V
+  uint64_t* s_full = v_empty + S;       // [2]
+  uint64_t* p_full = s_full + 2;        // [2]
+  uint64_t* pv_done = p_full + 2;       // one phase per P.V
+  uint64_t* o_done = pv_done + 1;
+  uint64_t* q_ready = o_done + 1;
+  uint64_t* drain = q_ready + 1;
 
-  if ((smem_u32(smem) & 1023u) != 0u) {  // SW128 boxes need a 1024-aligned base (uniform check)
-    if (threadIdx.x == 0) atomicOr(p.err, MFA_DEVERR_TIMEOUT);
-    return;
-  }
   if (threadIdx.x == 0) {
-    for (int st = 0; st < C::kStages; ++st) {
-      mbar_init(&full[st], 1);
-      mbar_init(&empty[st], kWarps);
+    for (int st = 0; st < S; ++st) {
+      mbar_init(&k_full[st], 1);
+      mbar_init(&k_empty[st], 1);
+      mbar_init(&v_full[st], 1);
+      mbar_init(&v_empty[st], 1);
     }
-    *sFlag = 0;
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 32);
+    }
+    mbar_init(pv_done, 1);
+    mbar_init(o_done, 1);
+    mbar_init(q_ready, 32);
+    mbar_init(drain, 1);
+    *s_abort = 0;
     fence_mbarrier_init();
   }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, C::kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
 
-  // ---- 1. the row's deduplicated list ----
+  // ---- 1. the row's deduplicated list (first occurrence kept) ----
   const int last = i + p.Nk - p.Nq;  // the row's position; keys after it are hidden
   const int32_t* lrow = p.sel + row_unit * p.sel_k;
-  int* sRaw = reinterpret_cast<int*>(smem + C::kS);  // scratch until the first scores
-  for (int e = threadIdx.x; e < p.sel_k; e += kThreads) sRaw[e] = lrow[e];
+  for (int e = threadIdx.x; e < p.sel_k; e += 128) sRaw[e] = lrow[e];
   __syncthreads();
-  {
-    const int e = threadIdx.x;  // sel_k <= kMaxSelK = 256 <= kThreads
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  int n_valid = 0;
+  for (int base = 0; base < p.sel_k; base += 128) {
+    const int e = base + threadIdx.x;
     bool keep = false;
     if (e < p.sel_k) {
       const int v = sRaw[e];
@@ -218,218 +157,261 @@ __global__ void __launch_bounds__(kWarpsFor<D, G> * 32, 1)
     const unsigned bal = __ballot_sync(0xffffffffu, keep);
     if (lane == 0) sCnt[warp] = __popc(bal);
     __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += sCnt[w];
-    if (keep) sList[base + __popc(bal & ((1u << lane) - 1u))] = sRaw[e];
-    if (threadIdx.x == 0) {
-      int tot = 0;
-      for (int w = 0; w < kWarps; ++w) tot += sCnt[w];
-      sCnt[16] = tot;
-    }
+    int off = n_valid;
+    for (int w = 0; w < warp; ++w) off += sCnt[w];
+    if (keep) sList[off + __popc(bal & ((1u << lane) - 1u))] = sRaw[e];
+    n_valid += sCnt[0] + sCnt[1] + sCnt[2] + sCnt[3];
     __syncthreads();
   }
-  const int n_valid = sCnt[16];
   const int per = (n_valid + p.n_split - 1) / p.n_split;
   const int j0 = min(part * per, n_valid), j1 = min(j0 + per, n_valid);
   const int nb = j1 - j0;
 
-  // ---- query rows in registers (packed pairs), in log2 units ----
-  uint64_t qr[G][DL / 2];
+  if (warp == 2) {
+    // =================== TMA producer ===================
+    // K and V of a block have their own barriers: K is released as soon as S
+    // of the block is done, V after its P.V, and the K loads run one block
+    // ahead of the V loads.
+    if (lane == 0) {
+      auto load = [&](const CUtensorMap* map, uint64_t* full, int n, int off) {
+        const int blk = sList[j0 + n];
+        mbar_arrive_expect_tx(full, C::kTile);
+        uint8_t* dst = smem + C::kStage0 + (n % S) * C::kStageBytes + off;
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const __nv_bfloat16* qp = p.q + b * p.qs0 + static_cast<int64_t>(g * G + h) * p.qs1 + i * p.qs2 + lane * DL;
-#pragma unroll
-    for (int e = 0; e < DL; e += 2) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(qp + e));
-      qr[h][e / 2] = f2_pack(f.x * p.scale_log2, f.y * p.scale_log2);
-    }
-  }
-  uint64_t acc[G][DL / 2];
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int e = 0; e < DL / 2; ++e) acc[h][e] = 0ull;  // +0.0f in both halves
-
-  auto issue = [&](int n) {  // thread 0: K and V of the part's n-th block into stage n % kStages
-    const int blk = sList[j0 + n], st = n % C::kStages;
-    mbar_arrive_expect_tx(&full[st], 2 * C::kTile);
-#pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      tma_load_4d(smem + C::kK + st * C::kTile + c * (kBlk * 128), &tm_k, &full[st], c * 64, blk * kBlk, g, b);
-      tma_load_4d(smem + C::kV + st * C::kTile + c * (kBlk * 128), &tm_v, &full[st], c * 64, blk * kBlk, g, b);
-    }
-  };
-  int n_issued = 0;  // thread 0's count of blocks whose loads went out
-  if (threadIdx.x == 0) {
-    n_issued = min(nb, C::kStages);
-    for (int n = 0; n < n_issued; ++n) issue(n);
-  }
-  int n_done = 0;  // blocks this warp has finished
-
-  // Per-warp online softmax: every warp keeps its own running max and sum of
-  // each query row (in every lane) and its own partial outputs, over the keys
-  // it handles; the warps are combined once after the last block. No
-  // block-wide barrier is needed per block: a stage is released by one
-  // arrival per warp, and thread 0 refills it when all have arrived.
-  float m_w[G], l_w[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    m_w[h] = -INFINITY;
-    l_w[h] = 0.f;
-  }
-  for (int n = 0; n < nb; ++n) {
-    const int st = n % C::kStages;
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (n / C::kStages) & 1, sFlag))) {
-      *sFlag = 1;
-      break;
-    }
-    const uint8_t* tK = smem + C::kK + st * C::kTile;
-    const uint8_t* tV = smem + C::kV + st * C::kTile;
-    const int kbase = sList[j0 + n] * kBlk;
-
-    // The warp's keys in chunks of kCk: scores, softmax update, P.V.
-#pragma unroll
-    for (int kc = 0; kc < kKeysPerWarp; kc += kCk) {
-    // ---- 3. scores of this chunk, gathered into every lane ----
-    float tot[kCk];
-#pragma unroll
-    for (int kk = 0; kk < kCk; ++kk) {
-      const int r = warp * kKeysPerWarp + kc + kk;
-      uint64_t kx[DL / 2];
-      load_row2<DL>(tK, r, lane, kx);
-      float part_dot[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        uint64_t s2 = f2_fma(qr[h][0], kx[0], 0ull);
-#pragma unroll
-        for (int e = 1; e < DL / 2; ++e) s2 = f2_fma(qr[h][e], kx[e], s2);
-        float lo, hi;
-        f2_unpack(s2, lo, hi);
-        part_dot[h] = lo + hi;
+        for (int c = 0; c < D / 64; ++c) tma_load_4d(dst + c * (kBlk * 128), map, full, c * 64, blk * kBlk, g, b);
+      };
+      int nk = 0, nv = 0;  // K and V loads issued
+      bool stop = false;
+      while (!stop && nv < nb) {
+        if (nk < nb && nk <= nv + 1) {
+          if (nk >= S && !mbar_wait(&k_empty[nk % S], ((nk / S) - 1) & 1, s_abort)) { stop = true; break; }
+          load(&tm_k, &k_full[nk % S], nk, C::kK);
+          ++nk;
+        } else {
+          if (nv >= S && !mbar_wait(&v_empty[nv % S], ((nv / S) - 1) & 1, s_abort)) { stop = true; break; }
+          load(&tm_v, &v_full[nv % S], nv, C::kV);
+          ++nv;
+        }
       }
-      tot[kk] = reduce_rows<G>(part_dot, lane);
+      if (*s_abort) {
+        volatile int no_abort = 0;
+        for (int j = (nk > S ? nk - S : 0); j < nk; ++j) mbar_wait(&k_full[j % S], (j / S) & 1, &no_abort);
+        for (int j = (nv > S ? nv - S : 0); j < nv; ++j) mbar_wait(&v_full[j % S], (j / S) & 1, &no_abort);
+      }
     }
-    float pk[G][kCk];
+  } else if (warp == 1) {
+    // =================== MMA issuer ===================
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, kBlk, false);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, true);
+    const uint32_t q_addr = smem_u32(smem + C::kQ), st_addr = smem_u32(smem + C::kStage0);
+    bool ok = true;
+    auto issue_s_ready = [&](int n) {
+      const int st = n % S;
+      tc_fence_after();
+      const uint32_t kb = st_addr + st * C::kStageBytes + C::kK;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      // ---- 4. online softmax of row h over these keys ----
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk & 3) * 32;
+        const uint32_t a = sdesc_sw128_lo(q_addr + (kk >> 2) * C::kQChunk + off, 16);
+        const uint32_t bd = sdesc_sw128_lo(kb + (kk >> 2) * (kBlk * 128) + off, 16);
+        umma_ss(tmem + (n & 1) * kBlk, a, bd, idesc_s, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(&s_full[n & 1]);
+      umma_commit(&k_empty[st]);
+    };
+    auto issue_pv = [&](int n) {
+      const int st = n % S;
+      tc_fence_after();
+      const uint32_t vd = sdesc_sw128_lo(st_addr + st * C::kStageBytes + C::kV, kBlk * 128);
+      const uint32_t a_p = tmem + (n & 1) * kBlk;
+#pragma unroll
+      for (int kk = 0; kk < kBlk / 16; ++kk)
+        umma_ts(tmem + 128, a_p + kk * 8, vd + kk * (16 * 128 / 16), idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(pv_done);
+      umma_commit(&v_empty[st]);
+    };
+    // Whichever is ready first goes out: the P.V of the oldest block whose P
+    // is written, or S of the next block once its K has landed and its S
+    // buffer is free (S(n) overwrites the P of block n - 2, so P.V(n - 2) must
+    // have gone out before it). A P.V never waits for the next block's data,
+    // so a stage is released, and refilled, as soon as its block is done.
+    int ns = 0, np = 0;  // S and P.V issued
+    uint64_t t_idle = 0;
+    while (ok && np < nb) {
+      bool did = false;
+      if (ns < nb && ns <= np + 1 && (ns > 0 || warp_all_dec(mbar_test_wait(q_ready, 0))) &&
+          warp_all_dec(mbar_test_wait(&k_full[ns % S], (ns / S) & 1))) {
+        issue_s_ready(ns);
+        ++ns;
+        did = true;
+      } else if (np < ns && warp_all_dec(mbar_test_wait(&p_full[np & 1], (np >> 1) & 1)) &&
+                 warp_all_dec(mbar_test_wait(&v_full[np % S], (np / S) & 1))) {
+        issue_pv(np);
+        ++np;
+        did = true;
+      }
+      if (did) {
+        t_idle = 0;
+      } else {
+        // Bounded like every other wait: give up after kWaitTimeoutNs without progress.
+        if (*s_abort) ok = false;
+        const uint64_t now = global_timer_ns();
+        if (t_idle == 0) t_idle = now;
+        else if (now - t_idle > kWaitTimeoutNs) ok = false;
+        ok = warp_all_dec(ok);
+      }
+    }
+    if (ok && nb > 0) umma_commit(o_done);
+    if (!ok) *s_abort = 1;
+    umma_commit(drain);
+    volatile int no_abort = 0;
+    mbar_wait(drain, 0, &no_abort);
+  } else if (warp == 0) {
+    // =================== Q, softmax, epilogue (lane h = query head h) ===================
+    const int h = lane;
+    const bool real = h < G;
+    // Q rows 0 .. G-1 into shared memory, K-major with the 128-byte swizzle
+    // (16-byte unit u of row h at u ^ (h & 7)), scaled later in the softmax.
+    if (real && nb > 0) {
+      const __nv_bfloat16* qrow = p.q + b * p.qs0 + static_cast<int64_t>(g * G + h) * p.qs1 + i * p.qs2;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 w = *reinterpret_cast<const uint4*>(qrow + c * 64 + u * 8);
+          st_shared_v4(smem_u32(smem + C::kQ + c * C::kQChunk + h * 128 + ((u ^ (h & 7)) << 4)), w.x, w.y, w.z, w.w);
+        }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(q_ready);
+    const uint32_t lane_off = 0;  // warp 0 reads TMEM lanes 0-31
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int n = 0; n < nb; ++n) {
+      const int kbase = sList[j0 + n] * kBlk;
+      if (!(ok = warp_all_dec(mbar_wait(&s_full[n & 1], (n >> 1) & 1, s_abort)))) break;
+      tc_fence_after();
+      float sc[kBlk];
+      {
+        uint32_t sv[2][32];
+        tmem_ld_32x32b_x32(tmem + lane_off + (n & 1) * kBlk, sv[0]);
+        tmem_ld_32x32b_x32(tmem + lane_off + (n & 1) * kBlk + 32, sv[1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < kBlk; ++jj) sc[jj] = __uint_as_float(sv[jj >> 5][jj & 31]);
+      }
+      // Keys after the row's position are hidden (this also covers the keys
+      // past Nk of a partial last block, which TMA fills with zeros).
+      const int vis = last - kbase + 1;  // visible keys of this block: [0, vis)
       float mx = -INFINITY;
 #pragma unroll
-      for (int kk = 0; kk < kCk; ++kk) {
-        const float v = __shfl_sync(0xffffffffu, tot[kk], owner_lane<G>(h));
-        pk[h][kk] = (kbase + warp * kKeysPerWarp + kc + kk <= last) ? v : -INFINITY;
-        mx = fmaxf(mx, pk[h][kk]);
+      for (int jj = 0; jj < kBlk; ++jj) {
+        if (jj >= vis) sc[jj] = -INFINITY;
+        mx = fmaxf(mx, sc[jj]);
       }
-      const float m_new = fmaxf(m_w[h], mx);
+      const float mx_s = mx * p.scale_log2;
+      const bool need = real && mx_s > m_run + 8.0f;
+      const float m_new = need ? mx_s : m_run;
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float alpha = ex2_approx(m_w[h] - m_use);  // 0 while nothing was visible
+      const float alpha = need ? ex2_approx(m_run - m_use) : 1.f;
+      uint32_t pk[kBlk / 2];
       float sum = 0.f;
 #pragma unroll
-      for (int kk = 0; kk < kCk; ++kk) {
-        pk[h][kk] = ex2_approx(pk[h][kk] - m_use);
-        sum += pk[h][kk];
+      for (int u = 0; u < kBlk / 2; ++u) {
+        const float e0 = ex2_approx(fmaf(sc[2 * u], p.scale_log2, -m_use));
+        const float e1 = ex2_approx(fmaf(sc[2 * u + 1], p.scale_log2, -m_use));
+        sum += e0 + e1;
+        pk[u] = pack_bf16x2(e0, e1);
       }
-      l_w[h] = l_w[h] * alpha + sum;
-      m_w[h] = m_new;
-      if (alpha != 1.f) {  // the same in every lane: no divergence
-        const uint64_t a2 = f2_pack(alpha, alpha);
+      l_run = l_run * alpha + sum;
+      m_run = m_new;
+      if (n > 0 && __any_sync(0xffffffffu, need)) {
+        // Rare: O has every P.V before this block's once pv_done's phase n - 1
+        // is complete (S of this block went out after that P.V).
+        if (!(ok = warp_all_dec(mbar_wait(pv_done, (n - 1) & 1, s_abort)))) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(tmem + lane_off + 128 + c * 32, o);
+          tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < DL / 2; ++e) acc[h][e] = f2_fma(acc[h][e], a2, 0ull);
+          for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+          tmem_st_32x32b_x32(tmem + lane_off + 128 + c * 32, o);
+        }
       }
-    }
-
-    // ---- 5. P.V of these keys ----
+      {
+        uint32_t a16[16], b16[16];
 #pragma unroll
-    for (int kk = 0; kk < kCk; ++kk) {
-      const int r = warp * kKeysPerWarp + kc + kk;
-      uint64_t vx[DL / 2];
-      load_row2<DL>(tV, r, lane, vx);
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const uint64_t p2 = f2_pack(pk[h][kk], pk[h][kk]);
-#pragma unroll
-        for (int e = 0; e < DL / 2; ++e) acc[h][e] = f2_fma(p2, vx[e], acc[h][e]);
+        for (int u = 0; u < 16; ++u) {
+          a16[u] = pk[u];
+          b16[u] = pk[16 + u];
+        }
+        tmem_st_32x32b_x16(tmem + lane_off + (n & 1) * kBlk, a16);
+        tmem_st_32x32b_x16(tmem + lane_off + (n & 1) * kBlk + 16, b16);
       }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[n & 1]);
     }
-    }  // key chunks
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[st]);
-    n_done = n + 1;
-    // Thread 0 refills stage st with block n + kStages once every warp has released it.
-    if (threadIdx.x == 0 && n + C::kStages < nb) {
-      if (mbar_wait(&empty[st], (n / C::kStages) & 1, sFlag)) {
-        issue(n + C::kStages);
-        n_issued = n + C::kStages + 1;
-      } else {
-        *sFlag = 1;
-      }
+    if (ok && nb > 0) {
+      ok = warp_all_dec(mbar_wait(o_done, 0, s_abort));
+      tc_fence_after();
     }
-  }
-  __syncthreads();
-  const bool aborted = *sFlag != 0;
-  if (aborted && threadIdx.x == 0) {
-    atomicOr(p.err, MFA_DEVERR_TIMEOUT);
-    // let the copies already issued land before shared memory is released
-    volatile int no_abort = 0;
-    for (int n = n_done; n < n_issued; ++n) mbar_wait(&full[n % C::kStages], (n / C::kStages) & 1, &no_abort);
-  }
-  if (aborted) return;
-
-  // ---- combine the warps (reusing the K/V ring and the score space) ----
-  // Rows of G * DL + 1 floats, so the 32 lanes' stores fall in different banks.
-  constexpr int kRow = G * DL + 1;
-  float* red = reinterpret_cast<float*>(smem + C::kK);   // [kWarps][32 lanes][kRow]
-  float* sMw = reinterpret_cast<float*>(smem + C::kS);    // [kWarps][G] running max
-  float* sLw = sMw + kWarps * G;                          // [kWarps][G] running sum
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int e = 0; e < DL / 2; ++e) {
-      float lo, hi;
-      f2_unpack(acc[h][e], lo, hi);
-      red[(warp * 32 + lane) * kRow + h * DL + 2 * e] = lo;
-      red[(warp * 32 + lane) * kRow + h * DL + 2 * e + 1] = hi;
-    }
-  if (lane == 0) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      sMw[warp * G + h] = m_w[h];
-      sLw[warp * G + h] = l_w[h];
-    }
-  }
-  __syncthreads();
-  // Element (h, dimension) = (h, DL * l + e) lives at lane l, slot h * DL + e of every warp.
-  for (int it = threadIdx.x; it < G * D; it += kThreads) {
-    const int h = it / D, d = it % D;
-    const int l = d / DL, e = d % DL;
-    float m = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, sMw[w * G + h]);
-    const float m_use = m == -INFINITY ? 0.f : m;
-    float o = 0.f, lsum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float wt = ex2_approx(sMw[w * G + h] - m_use);  // 0 for a warp that saw no key
-      o = fmaf(wt, red[(w * 32 + l) * kRow + h * DL + e], o);
-      lsum = fmaf(wt, sLw[w * G + h], lsum);
-    }
-    if (p.n_split == 1) {
-      const bool has = lsum > 0.f;
-      const float v = has ? o / lsum : 0.f;
-      __nv_bfloat16* orow = p.out + b * p.os0 + static_cast<int64_t>(g * G + h) * p.os1 + i * p.os2;
-      orow[d] = __float2bfloat16_rn(v);
-      if (d == 0)
-        p.lse[(static_cast<size_t>(b) * p.Hq + g * G + h) * p.Nq + i] =
-            has ? (m + __log2f(lsum)) * 0.69314718055994530942f : -INFINITY;
+    if (!ok) {
+      *s_abort = 1;
+      if (lane == 0) atomicOr(p.err, MFA_DEVERR_TIMEOUT);
     } else {
+      // ---- epilogue: head h's output row ----
+      const bool has = l_run > 0.f;
+      const float inv = has ? 1.f / l_run : 0.f;
       const size_t pu = row_unit * p.n_split + part;
-      p.o_part[(pu * G + h) * D + d] = o;
-      if (d == 0) {
-        // An empty part (or one that saw no visible key) carries m = -FLT_MAX, l = 0.
-        p.ml_part[(pu * G + h) * 2] = (m == -INFINITY) ? -FLT_MAX : m;
-        p.ml_part[(pu * G + h) * 2 + 1] = lsum;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (nb > 0) {
+          tmem_ld_32x32b_x32(tmem + lane_off + 128 + c * 32, o);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = 0u;
+        }
+        if (!real) continue;
+        if (p.n_split == 1) {
+          __nv_bfloat16* orow = p.out + b * p.os0 + static_cast<int64_t>(g * G + h) * p.os1 + i * p.os2 + c * 32;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              w[u] = pack_bf16x2(__uint_as_float(o[q4 * 8 + 2 * u]) * inv, __uint_as_float(o[q4 * 8 + 2 * u + 1]) * inv);
+            reinterpret_cast<uint4*>(orow)[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+          float* op = p.o_part + (pu * G + h) * D + c * 32;
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            reinterpret_cast<float4*>(op)[q4] =
+                make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]), __uint_as_float(o[4 * q4 + 2]),
+                            __uint_as_float(o[4 * q4 + 3]));
+        }
+      }
+      if (real) {
+        if (p.n_split == 1) {
+          p.lse[(static_cast<size_t>(b) * p.Hq + g * G + h) * p.Nq + i] =
+              has ? (m_run + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+        } else {
+          // A part that saw no visible key carries m = -FLT_MAX, l = 0.
+          p.ml_part[(pu * G + h) * 2] = m_run == -INFINITY ? -FLT_MAX : m_run;
+          p.ml_part[(pu * G + h) * 2 + 1] = l_run;
+        }
       }
     }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -496,12 +478,12 @@ mfa_status check_dec_tensor(const mfa_tensor* t) {
 
 template <int D, int G>
 mfa_status launch_dec(const CUtensorMap& mk, const CUtensorMap& mv, const DecParams& p, cudaStream_t s) {
-  using C = DecCfg<D>;
+  using C = DecTc<D>;
   static std::atomic<uint64_t> attr_devs{0};
   if (!ensure_smem_attr(reinterpret_cast<const void*>(mfa_decode_kernel<D, G>), C::kBytes, attr_devs))
     return MFA_ERR_CUDA;
   const dim3 grid(p.n_split, p.Nq, p.B * p.Hkv);
-  mfa_decode_kernel<D, G><<<grid, kWarpsFor<D, G> * 32, C::kBytes, s>>>(mk, mv, p);
+  mfa_decode_kernel<D, G><<<grid, 128, C::kBytes, s>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
   if (p.n_split > 1) {
     const dim3 cgrid(static_cast<unsigned>(p.B * p.Hkv * p.Nq), (G * D + kCombineThreads - 1) / kCombineThreads);
@@ -531,7 +513,7 @@ mfa_status launch_dec_g(const CUtensorMap& mk, const CUtensorMap& mv, const DecP
 int32_t auto_split(int64_t rows, int32_t sel_k, int D) {
   const int n_sm = device_sm_count();
   const int sms = n_sm > 0 ? n_sm : 148;
-  const int bytes = D == 128 ? DecCfg<128>::kBytes : DecCfg<256>::kBytes;
+  const int bytes = D == 128 ? DecTc<128>::kBytes : DecTc<256>::kBytes;
   const int per_sm = (227 * 1024) / bytes > 0 ? (227 * 1024) / bytes : 1;
   const int64_t target = (static_cast<int64_t>(sms) * per_sm * 85 + 99) / 100;
   const int64_t max_ns = sel_k / 2 > 1 ? sel_k / 2 : 1;
