@@ -351,9 +351,9 @@ mfa_status mfa_bwd(const mfa_tensor* q, const mfa_tensor* k, const mfa_tensor* v
                    const mfa_tensor* dk, const mfa_tensor* dv, void* workspace, size_t workspace_bytes,
                    void* stream);
 
-/* Bytes of the DEVICE workspace mfa_decode needs with n_split parts per list
- * (0 = the split mfa_decode chooses; 256 when no workspace is used; 0 on
- * invalid sizes). Host only. */
+/* Bytes of the DEVICE workspace mfa_decode needs for these sizes and n_split
+ * (0 = the automatic slot partition, which depends on the current device's SM
+ * count; 256 when no row is split; 0 on invalid sizes). Host only. */
 size_t mfa_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t Nq, int32_t D, int32_t sel_k,
                                   int32_t n_split);
 
@@ -372,12 +372,16 @@ size_t mfa_decode_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t Nq
  *   listed and j <= i + Nk - Nq (with Nq == Nk, the rule of MFA_MASK_BLOCKSEL).
  *   Rows that see no key get out = 0 and lse = -inf.
  *   lse     float32 [B, Hq, Nq] contiguous, natural log.
- *   n_split parts per list (0 = the fewest parts whose CTAs fill at least
- *           85 % of one wave on the SMs, at most sel_k / 2); with
- *           n_split > 1 the parts are combined by a second kernel (empty parts
- *           carry m = -FLT_MAX, so no exp(-inf - -inf) arises) and `workspace`
- *           (DEVICE, 256-byte aligned, mfa_decode_workspace_bytes bytes, owned
- *           by the caller) holds the partial results.
+ *   n_split how the lists are cut among CTAs. n_split >= 1: n_split parts of
+ *           ceil(sel_k / n_split) slots per list, one CTA each. 0: the lists
+ *           of all rows laid end to end and cut into equal slot ranges,
+ *           about one per SM (at least 2 slots, whole lists when a range
+ *           holds one or more), so a CTA may finish one row and start the
+ *           next. A row met by several CTAs is merged by a second kernel
+ *           (empty parts carry m = -FLT_MAX, so no exp(-inf - -inf) arises),
+ *           launched as a programmatic dependent of the first; `workspace`
+ *           (DEVICE, 256-byte aligned, mfa_decode_workspace_bytes bytes,
+ *           owned by the caller) then holds the partial results.
  *   dev_err DEVICE uint32 the kernels OR MFA_DEVERR_* bits into (required; the
  *           caller clears it).
  * Errors: MFA_ERR_INVALID_ARG, MFA_ERR_SHAPE_MISMATCH, MFA_ERR_UNSUPPORTED

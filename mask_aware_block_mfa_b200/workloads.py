@@ -387,6 +387,18 @@ def make_decode_problem(name: str):
     return q, k, v, sel
 
 
+def decode_selection_sets(name: str, count: int) -> list:
+    """`count` selection arrays for a decode workload: the workload's own first,
+    then lists drawn the same way from further seeds. Timed steps cycle through
+    them, so that the blocks a step reads were not read by the step before."""
+    B, Hq, Hkv, Nq, Nk, d, sel_k = DECODE_SHAPES[name]
+    seed = DECODE_SEEDS[name]
+    out = [make_decode_problem(name)[3]]
+    for r in range(1, count):
+        out.append(decode_selection(np.random.default_rng(seed + 1000 * r), B, Hkv, Nq, Nk, sel_k))
+    return out
+
+
 def random_colwise(rng: np.random.Generator, B: int, Hm: int, Nq: int, Nk: int,
                    p_empty: float = 0.3) -> MaskDesc:
     """Arbitrary column bounds in [0, Nq] (empty intervals included) for stress tests."""

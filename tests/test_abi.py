@@ -274,6 +274,29 @@ def test_decode_rejects_bad_arguments_on_host(lib):
     assert call(q=f32) == B.MFA_ERR_UNSUPPORTED
 
 
+def _ws(rows, seg, G, D):
+    up = lambda x: -(-x // 256) * 256
+    return up(rows * seg * G * D * 4) + up(rows * seg * G * 2 * 4)
+
+
+def test_decode_workspace_follows_the_slot_partition(lib):
+    """The automatic split gives each CTA ceil(rows * sel_k / SMs) of the rows'
+    list slots laid end to end (148 SMs: a B200, and the count used without a
+    device), widened to a divisor of sel_k while three quarters of the SMs
+    stay busy. decode_sel64k: 64 lists of 32 slots, 14 -> 16 slots per CTA,
+    128 CTAs, 2 partials per row. 20 lists of 40 slots: 6 slots per CTA (the
+    divisor 8 would leave 100 CTAs), so a row meets up to ceil(39 / 6) + 1 = 8
+    CTAs. 2000 lists of 256 slots: a CTA takes whole lists (8 at most) and no
+    row is split: no workspace. An explicit n_split keeps n_split partials
+    per row, none for 1."""
+    assert lib.mfa_decode_workspace_bytes(8, 32, 8, 1, 256, 32, 0) == _ws(64, 2, 4, 256)
+    assert lib.mfa_decode_workspace_bytes(2, 8, 2, 5, 256, 40, 0) == _ws(20, 8, 4, 256)
+    assert lib.mfa_decode_workspace_bytes(1, 4, 2, 1000, 128, 256, 0) == 256
+    assert lib.mfa_decode_workspace_bytes(8, 32, 8, 1, 256, 32, 1) == 256
+    assert lib.mfa_decode_workspace_bytes(8, 32, 8, 1, 256, 32, 3) == _ws(64, 3, 4, 256)
+    assert lib.mfa_decode_workspace_bytes(1, 8, 2, 0, 256, 16, 0) == 256     # no rows
+
+
 def test_fwd_bias_rejects_bad_arguments_on_host(lib):
     m = _fake_map(lib)
     q, k, v, o = _fake_tensor(1, 8, 512, 128), _fake_tensor(1, 2, 512, 128), _fake_tensor(1, 2, 512, 128), \

@@ -43,6 +43,8 @@ CASES = [
     (128, 1, 4, 777, 20, 3),
     (256, 2, 16, 2000, 40, 0),
     (128, 8, 70, 64, 4, 2),     # rows 0..5 sit before the sequence start: no key
+    (256, 4, 5, 3000, 40, 0),   # 20 rows of 40 slots, 6 per CTA: rows split over up to 8 CTAs
+    (128, 2, 300, 2500, 8, 0),  # 1200 rows of 8 slots: every CTA takes 9 whole rows, no partials
 ]
 
 
@@ -113,3 +115,16 @@ def test_decode_longest_lists():
         out, lse, err = run(q, k, v, sel, n_split)
         assert err == 0
         compare_attention(out, lse, *ref)
+
+
+def test_decode_slot_ranges_over_many_rows_and_waves():
+    """2000 rows of 256 slots (at most 64 blocks in a 4096-key cache, so most
+    slots are pads or duplicates): the automatic split gives every CTA 8 whole
+    rows, 250 CTAs in two waves; one row in 7 is compared (the oracle is the
+    given the same rows)."""
+    q, k, v, sel = _inputs(11, 1, 4, 2, 1000, 4096, 128, 256, pads=100, dups=40)
+    out, lse, err = run(q, k, v, sel)
+    assert err == 0
+    rows = list(range(0, 1000, 7))
+    ref_out, ref_lse = OD.decode_attention(q, k, v, sel, rows=rows)
+    compare_attention(out[:, :, rows], lse[:, :, rows], ref_out, ref_lse)
