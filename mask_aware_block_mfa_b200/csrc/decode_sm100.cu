@@ -65,10 +65,12 @@ __device__ __forceinline__ bool warp_all_dec(bool ok) { return __all_sync(0xffff
 // ---------------------------------------------------------------------------
 // The decode kernel on the tensor cores.
 //
-// S = Q K^T as one tcgen05 MMA of M = 128 rows: rows 0 .. G-1 are the G query
-// heads of the row, the other rows of the A operand read whatever follows Q in
-// shared memory and their results are never used, so Q takes 16 rows (2 KB) per
-// 64-column chunk instead of 128. N = 64 keys (one block), K = D. Lane h of the
+// S = Q K^T as one tcgen05 MMA of M = 128 rows with Q in TMEM (the TS form):
+// lanes 0 .. G-1 hold the G query heads of the row, lanes G .. 31 zeros, and
+// the results of the other lanes are never used. N = 64 keys (one block), K =
+// D. With Q and P in TMEM, the tensor core reads only K and V from shared
+// memory, once each: shared-memory bandwidth (TMA writes plus MMA operand
+// reads) is what bounds a block's turn-around. Lane h of the
 // softmax warp holds head h's 64 scores (TMEM lane = row), keeps its own
 // online max and sum, and writes P (bf16) over its scores. O += P V as a TS
 // MMA (P from TMEM) with N = D, into an accumulator of 128 x D fp32 columns.
@@ -80,10 +82,11 @@ __device__ __forceinline__ bool warp_all_dec(bool ok) { return __all_sync(0xffff
 //
 // A CTA's blocks form one stream across its rows (segments): the ring, the S
 // buffers and the MMA order run on from one row into the next. Q arrives by
-// TMA into one of two buffers, so the next row's Q loads while this row's S
-// products still read the other. The first P.V of a row overwrites O; it
-// follows the softmax warp's P of that row's first block, which the warp
-// writes only after it has read the previous row's O.
+// TMA into one of two shared-memory buffers ahead of its row; the softmax
+// warp copies it into TMEM when the previous row's S products are done (it
+// has waited for the last of them) and releases the buffer. The first P.V
+// of a row overwrites O; it follows the softmax warp's P of that row's first
+// block, which the warp writes only after it has read the previous row's O.
 //
 // Warps: 0 softmax and epilogue (TMEM lanes 0-31), 1 MMA issuer and TMEM owner,
 // 2 TMA producer, 3 idle. Every wait is bounded.
@@ -101,13 +104,14 @@ struct DecTc {
   static constexpr int kRaw = kStage0 + kStages * kStageBytes;  // one row's raw list [kMaxSelK]
   static constexpr int kList = kRaw + kMaxSelK * 4;             // the CTA's kept blocks [kMaxPer]
   static constexpr int kSeg = kList + kMaxPer * 4;              // segment starts in the kept list [kMaxSeg + 1]
-  static constexpr int kMisc = kSeg + ((kMaxSeg + 1) * 4 + 15) / 16 * 16;
+  static constexpr int kCoord = kSeg + ((kMaxSeg + 1) * 4 + 15) / 16 * 16;  // (b, g, i) per segment [kMaxSeg]
+  static constexpr int kMisc = kCoord + kMaxSeg * 16;
   static constexpr int kBytes = kMisc + 512 + 1024;         // + slack for 1024-byte alignment
-  static constexpr int kTmemCols = 128 + D <= 256 ? 256 : 512;  // S0 [0,64) S1 [64,128) O [128, 128 + D)
+  static constexpr int kTmemCols = 512;        // S0 [0,64) S1 [64,128) O [128, 128 + D) Q [128 + D, 128 + 3D/2)
+  static constexpr int kQCol = 128 + D;
   static_assert(kBytes <= 232448, "shared memory");
   static_assert(2 * kQBytes <= kStage0, "Q buffers");
-  // M = 128 reads 16 KB from each Q chunk's base: the last one must stay inside the allocation.
-  static_assert(kQBytes + (D / 64 - 1) * kQChunk + 16 * 1024 <= kRaw, "Q chunk rows beyond 16 read allocated memory");
+  static_assert(kQCol + D / 2 <= kTmemCols, "TMEM columns");
 };
 
 template <int D, int G>
@@ -128,6 +132,7 @@ __global__ void __launch_bounds__(128, 1)
   int* sRaw = reinterpret_cast<int*>(smem + C::kRaw);
   int* sList = reinterpret_cast<int*>(smem + C::kList);
   int* sSeg = reinterpret_cast<int*>(smem + C::kSeg);            // row k's blocks: sList[sSeg[k] .. sSeg[k + 1])
+  int4* sCoord = reinterpret_cast<int4*>(smem + C::kCoord);     // row k's (b, g, i)
   int* sCnt = reinterpret_cast<int*>(smem + C::kMisc);          // [4] per-warp counts
   volatile int* s_abort = reinterpret_cast<volatile int*>(sCnt + 8);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sCnt + 9);
@@ -136,9 +141,10 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t* k_empty = k_full + S;       // [S]: S of the block is done with K
   uint64_t* v_full = k_empty + S;       // [S]
   uint64_t* v_empty = v_full + S;       // [S]: P.V of the block is done with V
-  uint64_t* q_full = v_empty + S;       // [2]
-  uint64_t* q_empty = q_full + 2;       // [2]: the row's last S is done with its Q
-  uint64_t* s_full = q_empty + 2;       // [2]
+  uint64_t* q_full = v_empty + S;       // [2]: Q of a row in shared memory
+  uint64_t* q_empty = q_full + 2;       // [2]: copied into TMEM, the buffer is free
+  uint64_t* q_ready = q_empty + 2;      // Q of the next row with blocks is in TMEM
+  uint64_t* s_full = q_ready + 1;       // [2]
   uint64_t* p_full = s_full + 2;        // [2]
   uint64_t* pv_done = p_full + 2;       // one phase per P.V
   uint64_t* o_done = pv_done + 1;       // one phase per row with blocks
@@ -160,6 +166,7 @@ __global__ void __launch_bounds__(128, 1)
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 32);
     }
+    mbar_init(q_ready, 1);
     mbar_init(pv_done, 1);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
@@ -182,7 +189,11 @@ __global__ void __launch_bounds__(128, 1)
     const int ea = static_cast<int>(a < 0 ? 0 : (a < p.sel_k ? a : p.sel_k));
     const int eb = static_cast<int>(e < p.sel_k ? e : p.sel_k);
     const int last = static_cast<int>(r % p.Nq) + p.Nk - p.Nq;  // the row's position
-    if (threadIdx.x == 0) sSeg[k] = total;
+    if (threadIdx.x == 0) {
+      sSeg[k] = total;
+      const int64_t bg = r / p.Nq;
+      sCoord[k] = make_int4(static_cast<int>(bg / p.Hkv), static_cast<int>(bg % p.Hkv), static_cast<int>(r % p.Nq), 0);
+    }
     if (eb <= ea) continue;
     const int32_t* lrow = p.sel + r * p.sel_k;
     for (int e = threadIdx.x; e < eb; e += 128) sRaw[e] = lrow[e];
@@ -224,15 +235,11 @@ __global__ void __launch_bounds__(128, 1)
     // of the block is done, V after its P.V, and the K loads run one block
     // ahead of the V loads. A row's Q goes out just before its first K.
     if (lane == 0) {
-      auto coords = [&](int64_t r, int& b, int& g, int& i) {
-        const int64_t bg = r / p.Nq;
-        i = static_cast<int>(r % p.Nq);
-        b = static_cast<int>(bg / p.Hkv);
-        g = static_cast<int>(bg % p.Hkv);
-      };
+      // The row's coordinates come from shared memory: 64-bit divisions here
+      // would sit on the issue path of every load.
       auto load = [&](const CUtensorMap* map, uint64_t* full, int n, int off, int seg) {
-        int b, g, i;
-        coords(r0 + seg, b, g, i);
+        const int4 co = sCoord[seg];
+        const int b = co.x, g = co.y;
         const int blk = sList[n];
         mbar_arrive_expect_tx(full, C::kTile);
         uint8_t* dst = smem + C::kStage0 + (n % S) * C::kStageBytes + off;
@@ -248,8 +255,8 @@ __global__ void __launch_bounds__(128, 1)
           if (nk == sSeg[kseg]) {
             // Q buffer nq & 1 is free once the S products of row nq - 2 are done.
             if (nq >= 2 && !mbar_wait(&q_empty[nq & 1], ((nq >> 1) - 1) & 1, s_abort)) { stop = true; break; }
-            int b, g, i;
-            coords(r0 + kseg, b, g, i);
+            const int4 co = sCoord[kseg];
+            const int b = co.x, g = co.y, i = co.z;
             mbar_arrive_expect_tx(&q_full[nq & 1], G * 128 * (D / 64));
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
@@ -279,24 +286,20 @@ __global__ void __launch_bounds__(128, 1)
     // =================== MMA issuer ===================
     constexpr uint32_t idesc_s = idesc_bf16_f32(128, kBlk, false);
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, true);
-    const uint32_t q_addr = smem_u32(smem + C::kQ), st_addr = smem_u32(smem + C::kStage0);
+    const uint32_t st_addr = smem_u32(smem + C::kStage0);
     bool ok = true;
     int sseg = 0, sq = 0, pseg = 0, pq = 0;  // rows of the next S and the next P.V
     auto issue_s_ready = [&](int n) {
       const int st = n % S;
       tc_fence_after();
-      const uint32_t qb = q_addr + (sq & 1) * C::kQBytes;
       const uint32_t kb = st_addr + st * C::kStageBytes + C::kK;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk & 3) * 32;
-        const uint32_t a = sdesc_sw128_lo(qb + (kk >> 2) * C::kQChunk + off, 16);
-        const uint32_t bd = sdesc_sw128_lo(kb + (kk >> 2) * (kBlk * 128) + off, 16);
-        umma_ss(tmem + (n & 1) * kBlk, a, bd, idesc_s, kk > 0 ? 1u : 0u);
+        const uint32_t bd = sdesc_sw128_lo(kb + (kk >> 2) * (kBlk * 128) + (kk & 3) * 32, 16);
+        umma_ts(tmem + (n & 1) * kBlk, tmem + C::kQCol + kk * 8, bd, idesc_s, kk > 0 ? 1u : 0u);
       }
       umma_commit(&s_full[n & 1]);
       umma_commit(&k_empty[st]);
-      if (n + 1 == sSeg[sseg + 1]) umma_commit(&q_empty[sq & 1]);
     };
     auto issue_pv = [&](int n) {
       const int st = n % S;
@@ -313,7 +316,7 @@ __global__ void __launch_bounds__(128, 1)
     };
     // Whichever is ready first goes out: the P.V of the oldest block whose P
     // is written, or S of the next block once its K (and, for a row's first
-    // block, its Q) has landed and its S buffer is free (S(n) overwrites the P
+    // block, its Q in TMEM) is there and its S buffer is free (S(n) overwrites the P
     // of block n - 2, so P.V(n - 2) must have gone out before it). A P.V never
     // waits for the next block's data, so a stage is released, and refilled,
     // as soon as its block is done.
@@ -323,7 +326,7 @@ __global__ void __launch_bounds__(128, 1)
       bool did = false;
       if (ns < total && ns <= np + 1) {
         seek(ns, sseg, sq);
-        if ((ns != sSeg[sseg] || warp_all_dec(mbar_test_wait(&q_full[sq & 1], (sq >> 1) & 1))) &&
+        if ((ns != sSeg[sseg] || warp_all_dec(mbar_test_wait(q_ready, sq & 1))) &&
             warp_all_dec(mbar_test_wait(&k_full[ns % S], (ns / S) & 1))) {
           issue_s_ready(ns);
           ++ns;
@@ -368,6 +371,35 @@ __global__ void __launch_bounds__(128, 1)
       const int last = i + p.Nk - p.Nq;
       const int nb = sSeg[k + 1] - sSeg[k];
       float m_run = -INFINITY, l_run = 0.f;
+      if (nb > 0) {
+        // Q of this row into TMEM lanes 0-31 (lane h: head h, zeros past G).
+        // Every S product of the previous row is done: this warp has waited
+        // for the last one.
+        const int qb = rows_done & 1;
+        if (!(ok = warp_all_dec(mbar_wait(&q_full[qb], (rows_done >> 1) & 1, s_abort)))) break;
+        const uint8_t* qrow = smem + C::kQ + qb * C::kQBytes + lane * 128;
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t w[32];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            uint4 x = make_uint4(0u, 0u, 0u, 0u);
+            if (real) x = *reinterpret_cast<const uint4*>(qrow + c * C::kQChunk + ((u ^ (lane & 7)) << 4));
+            w[4 * u] = x.x;
+            w[4 * u + 1] = x.y;
+            w[4 * u + 2] = x.z;
+            w[4 * u + 3] = x.w;
+          }
+          tmem_st_32x32b_x32(tmem + lane_off + C::kQCol + c * 32, w);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(q_ready);
+          mbar_arrive(&q_empty[qb]);
+        }
+      }
       for (int t = 0; t < nb; ++t, ++n) {
         const int kbase = sList[n] * kBlk;
         if (!(ok = warp_all_dec(mbar_wait(&s_full[n & 1], (n >> 1) & 1, s_abort)))) break;
