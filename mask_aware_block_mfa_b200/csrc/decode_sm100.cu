@@ -102,7 +102,7 @@ struct DecTc {
   static constexpr int kK = 0, kV = kTile;                   // inside a stage
   static constexpr int kStageBytes = 2 * kTile;
   static constexpr int kRaw = kStage0 + kStages * kStageBytes;  // one row's raw list [kMaxSelK]
-  static constexpr int kList = kRaw + kMaxSelK * 4;             // the CTA's kept blocks [kMaxPer]
+  static constexpr int kList = kRaw + kMaxSelK * 4 + 16;        // the CTA's kept blocks [kMaxPer]
   static constexpr int kSeg = kList + kMaxPer * 4;              // segment starts in the kept list [kMaxSeg + 1]
   static constexpr int kCoord = kSeg + ((kMaxSeg + 1) * 4 + 15) / 16 * 16;  // (b, g, i) per segment [kMaxSeg]
   static constexpr int kMisc = kCoord + kMaxSeg * 16;
@@ -150,6 +150,16 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t* o_done = pv_done + 1;       // one phase per row with blocks
   uint64_t* drain = o_done + 1;
 
+  // The first row's list is read before anything else, so that the latency
+  // of that global load overlaps the barrier and TMEM set-up below.
+  int pre0 = -1, pre1 = -1;
+  {
+    const int64_t e = v1 - r0 * p.L;
+    const int eb0 = static_cast<int>(e < p.sel_k ? e : p.sel_k);
+    const int32_t* lrow0 = p.sel + r0 * p.sel_k;
+    if (static_cast<int>(threadIdx.x) < eb0) pre0 = __ldg(lrow0 + threadIdx.x);
+    if (static_cast<int>(threadIdx.x) + 128 < eb0) pre1 = __ldg(lrow0 + threadIdx.x + 128);
+  }
   // The combine kernel (a programmatic dependent launch) may be scheduled now:
   // it waits for this grid to complete before it reads anything.
   asm volatile("griddepcontrol.launch_dependents;");
@@ -196,7 +206,15 @@ __global__ void __launch_bounds__(128, 1)
     }
     if (eb <= ea) continue;
     const int32_t* lrow = p.sel + r * p.sel_k;
-    for (int e = threadIdx.x; e < eb; e += 128) sRaw[e] = lrow[e];
+    if (k == 0) {
+      if (static_cast<int>(threadIdx.x) < eb) sRaw[threadIdx.x] = pre0;
+      if (static_cast<int>(threadIdx.x) + 128 < eb) sRaw[threadIdx.x + 128] = pre1;
+    } else {
+      for (int e = threadIdx.x; e < eb; e += 128) sRaw[e] = lrow[e];
+    }
+    // Entries up to the next multiple of 4 past eb are padding for the
+    // vector compares below (never equal to a kept entry: -2).
+    if (static_cast<int>(threadIdx.x) < 4) sRaw[eb + threadIdx.x] = -2;
     __syncthreads();
     for (int base = ea; base < eb; base += 128) {
       const int e = base + threadIdx.x;
@@ -205,7 +223,17 @@ __global__ void __launch_bounds__(128, 1)
         const int v = sRaw[e];
         if (v < -1 || v >= p.nblk) atomicOr(p.err, MFA_DEVERR_SEL);
         keep = v >= 0 && v < p.nblk && static_cast<int64_t>(v) * kBlk <= last;
-        for (int e2 = 0; keep && e2 < e; ++e2) keep = sRaw[e2] != v;
+        // First occurrence: no equal entry before e. Four entries per
+        // shared-memory load and no early exit, so the loads pipeline.
+        if (keep) {
+          const int4* raw4 = reinterpret_cast<const int4*>(sRaw);
+          bool dup = false;
+          for (int e2 = 0; e2 < e; e2 += 4) {
+            const int4 w = raw4[e2 >> 2];
+            dup |= (w.x == v) | ((w.y == v) & (e2 + 1 < e)) | ((w.z == v) & (e2 + 2 < e)) | ((w.w == v) & (e2 + 3 < e));
+          }
+          keep = !dup;
+        }
       }
       const unsigned bal = __ballot_sync(0xffffffffu, keep);
       if (lane == 0) sCnt[warp] = __popc(bal);
