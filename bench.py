@@ -548,18 +548,24 @@ def run_decode(args, rank, world, local):
         step(seld_all[w % DECODE_SETS])
     if dec.status() != 0:
         raise RuntimeError("device error bits set during warm-up")
-    graphs = []
+    # One CUDA graph holds DECODE_SETS steps (one per selection set), as a
+    # serving loop captures its decode calls together; one-step graphs cover
+    # a remainder of K.
     cap = torch.cuda.Stream(dev)
-    for sd in seld_all:
+
+    def capture(fn):
         graph = torch.cuda.CUDAGraph()
         cap.wait_stream(stream)
         with torch.cuda.stream(cap):
             with torch.cuda.graph(graph, stream=cap):
-                step(sd)
+                fn()
         stream.wait_stream(cap)
-        graphs.append(graph)
-    for w in range(max(args.warmup, DECODE_SETS)):
-        graphs[w % DECODE_SETS].replay()
+        return graph
+
+    graphs = [capture(lambda sd=sd: step(sd)) for sd in seld_all]
+    graph_all = capture(lambda: [step(sd) for sd in seld_all])
+    for w in range(max(args.warmup, 1)):
+        graph_all.replay()
     torch.cuda.synchronize(dev)
     # The K steps run back to back between two events, as a serving loop runs
     # them (no flush is needed between them: see DECODE_SETS above).
@@ -570,8 +576,10 @@ def run_decode(args, rank, world, local):
     with ClockSampler(local) as clk:
         time.sleep(0.3)
         e0.record(stream)
-        for st in range(args.steps):
-            graphs[st % DECODE_SETS].replay()
+        for _ in range(args.steps // DECODE_SETS):
+            graph_all.replay()
+        for st in range(args.steps % DECODE_SETS):
+            graphs[st].replay()
         e1.record(stream)
         torch.cuda.synchronize(dev)
         time.sleep(0.2)
@@ -619,7 +627,9 @@ def run_decode(args, rank, world, local):
                    "l2": f"inputs larger than L2: no flush; the steps cycle through {DECODE_SETS} seeded selection "
                          "sets, so a step's blocks were last read that many steps earlier",
                    "timing": "the K steps back to back between two CUDA events",
-                   "parallelism": f"replicas x{world}", "launch": "each step replayed as a CUDA graph"},
+                   "parallelism": f"replicas x{world}",
+                   "launch": f"CUDA graphs of {DECODE_SETS} steps (one per selection set), one-step graphs for a "
+                             "remainder of K"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": ncu_traffic(args.workload, DEC_NCU_TRAFFIC, DEC_KERNEL_SOURCES),
                      "peak_kind": f"{src} HBM copy bandwidth; achieved over the decode call (decode + combine), "
