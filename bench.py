@@ -70,15 +70,15 @@ NCU_TRAFFIC = {
 BWD_KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/bwd_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh",
                       "mask_aware_block_mfa_b200/csrc/order.cuh")
 BWD_NCU_TRAFFIC = {
-    "doc8k": (842_567_936, "f7dbd95ed2e4419e"),
-    "doc32k": (2_108_606_464, "f7dbd95ed2e4419e"),
+    "doc8k": (851_308_032, "542bc078d317add5"),
+    "doc32k": (2_108_781_056, "542bc078d317add5"),
 }
 
 
 # The same for the decode kernel (mfa_decode_kernel) of --pass decode.
 DEC_KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/decode_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh")
 DEC_NCU_TRAFFIC = {
-    "decode_sel64k": (138_585_600, "53beade334f441f6"),
+    "decode_sel64k": (137_548_544, "0f12f154345792bb"),
 }
 
 
