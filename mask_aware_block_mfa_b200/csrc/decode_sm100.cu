@@ -35,6 +35,7 @@ namespace {
 
 constexpr int kBlk = 64;       // keys per selection block
 constexpr int kCombineThreads = 256;
+constexpr int kCombineFast = 8;  // partials per row merged with all loads in one round
 constexpr int kMaxPer = 2048;  // list slots per CTA
 constexpr int kMaxSeg = 64;    // rows (segments) per CTA
 
@@ -507,17 +508,8 @@ __global__ void __launch_bounds__(128, 1)
       const bool has = l_run > 0.f;
       const float inv = has ? 1.f / l_run : 0.f;
       const size_t pu = static_cast<size_t>(r) * p.seg_max + (blockIdx.x - first_cta(p, r));
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (nb > 0) {
-          tmem_ld_32x32b_x32(tmem + lane_off + 128 + c * 32, o);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int u = 0; u < 32; ++u) o[u] = 0u;
-        }
-        if (!real) continue;
+      // Two 32-column TMEM loads per wait: the epilogue is on the CTA's tail.
+      auto emit = [&](const uint32_t (&o)[32], int c) {
         if (whole) {
           __nv_bfloat16* orow = p.out + b * p.os0 + static_cast<int64_t>(g * G + h) * p.os1 + i * p.os2 + c * 32;
 #pragma unroll
@@ -536,6 +528,21 @@ __global__ void __launch_bounds__(128, 1)
                 make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]), __uint_as_float(o[4 * q4 + 2]),
                             __uint_as_float(o[4 * q4 + 3]));
         }
+      };
+#pragma unroll 1
+      for (int c = 0; c < D / 32; c += 2) {
+        uint32_t o0[32], o1[32];
+        if (nb > 0) {
+          tmem_ld_32x32b_x32(tmem + lane_off + 128 + c * 32, o0);
+          tmem_ld_32x32b_x32(tmem + lane_off + 128 + (c + 1) * 32, o1);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o0[u] = o1[u] = 0u;
+        }
+        if (!real) continue;
+        emit(o0, c);
+        emit(o1, c + 1);
       }
       if (real) {
         if (whole) {
@@ -583,14 +590,38 @@ __global__ void __launch_bounds__(kCombineThreads) mfa_decode_combine(const DecP
   if (it < G * D) {
     const int h = it / D, d = it % D;
     const size_t pu0 = static_cast<size_t>(ru) * p.seg_max;
-    float M = -FLT_MAX;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, p.ml_part[((pu0 + s) * G + h) * 2]);
-    float o = 0.f, l = 0.f;
-    for (int s = 0; s < ns; ++s) {
-      const size_t pu = pu0 + s;
-      const float w = ex2_approx(p.ml_part[(pu * G + h) * 2] - M);
-      o = fmaf(w, p.o_part[(pu * G + h) * D + d], o);
-      l = fmaf(w, p.ml_part[(pu * G + h) * 2 + 1], l);
+    float M = -FLT_MAX, o = 0.f, l = 0.f;
+    if (ns <= kCombineFast) {
+      // Every load goes out before any is used: one round of L2 latency.
+      float mv[kCombineFast], lv[kCombineFast], ov[kCombineFast];
+#pragma unroll
+      for (int s = 0; s < kCombineFast; ++s) {
+        if (s < ns) {
+          const size_t pu = pu0 + s;
+          mv[s] = p.ml_part[(pu * G + h) * 2];
+          lv[s] = p.ml_part[(pu * G + h) * 2 + 1];
+          ov[s] = p.o_part[(pu * G + h) * D + d];
+        }
+      }
+#pragma unroll
+      for (int s = 0; s < kCombineFast; ++s)
+        if (s < ns) M = fmaxf(M, mv[s]);
+#pragma unroll
+      for (int s = 0; s < kCombineFast; ++s) {
+        if (s < ns) {
+          const float w = ex2_approx(mv[s] - M);
+          o = fmaf(w, ov[s], o);
+          l = fmaf(w, lv[s], l);
+        }
+      }
+    } else {
+      for (int s = 0; s < ns; ++s) M = fmaxf(M, p.ml_part[((pu0 + s) * G + h) * 2]);
+      for (int s = 0; s < ns; ++s) {
+        const size_t pu = pu0 + s;
+        const float w = ex2_approx(p.ml_part[(pu * G + h) * 2] - M);
+        o = fmaf(w, p.o_part[(pu * G + h) * D + d], o);
+        l = fmaf(w, p.ml_part[(pu * G + h) * 2 + 1], l);
+      }
     }
     const bool has = l > 0.f;
     __nv_bfloat16* orow = p.out + b * p.os0 + static_cast<int64_t>(g * G + h) * p.os1 + i * p.os2;
