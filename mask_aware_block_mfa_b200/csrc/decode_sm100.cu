@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(128, 1)
   int* sCnt = reinterpret_cast<int*>(smem + C::kMisc);          // [4] per-warp counts
   volatile int* s_abort = reinterpret_cast<volatile int*>(sCnt + 8);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sCnt + 9);
+  int* s_early = sCnt + 10;                                     // Q, K, V of block 0 issued before the roles
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kMisc + 64);
   uint64_t* k_full = bars;              // [S]
   uint64_t* k_empty = k_full + S;       // [S]: S of the block is done with K
@@ -183,6 +184,42 @@ __global__ void __launch_bounds__(128, 1)
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_mbarrier_init();
+  }
+  // The first block's loads go out before the deduplication when the first
+  // slot of the CTA's range is a kept block of the first row: valid, at or
+  // before the row's position, and not listed earlier in the row (its
+  // earlier entries, fewer than 32, are in warp 0's registers). It is then
+  // the first entry of the kept list, and the producer starts at block 1.
+  if (warp == 0) {
+    const int64_t a = v0 - r0 * p.L, e = v1 - r0 * p.L;
+    const int ea0 = static_cast<int>(a < 0 ? 0 : (a < p.sel_k ? a : p.sel_k));
+    const int eb0 = static_cast<int>(e < p.sel_k ? e : p.sel_k);
+    int early = -1;
+    if (ea0 < 32 && ea0 < eb0) {
+      const int vf = __shfl_sync(0xffffffffu, pre0, ea0);
+      const bool dup = __ballot_sync(0xffffffffu, lane < ea0 && pre0 == vf) != 0u;
+      const int last0 = static_cast<int>(r0 % p.Nq) + p.Nk - p.Nq;
+      if (!dup && vf >= 0 && vf < p.nblk && static_cast<int64_t>(vf) * kBlk <= last0) early = vf;
+    }
+    if (lane == 0) {
+      *s_early = early >= 0 ? 1 : 0;
+      if (early >= 0) {
+        const int64_t bg = r0 / p.Nq;
+        const int b = static_cast<int>(bg / p.Hkv), g = static_cast<int>(bg % p.Hkv), i = static_cast<int>(r0 % p.Nq);
+        mbar_arrive_expect_tx(&q_full[0], G * 128 * (D / 64));
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(smem + C::kQ + c * C::kQChunk, &tm_q, &q_full[0], c * 64, i, g * G, b);
+        mbar_arrive_expect_tx(&k_full[0], C::kTile);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(smem + C::kStage0 + C::kK + c * (kBlk * 128), &tm_k, &k_full[0], c * 64, early * kBlk, g, b);
+        mbar_arrive_expect_tx(&v_full[0], C::kTile);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(smem + C::kStage0 + C::kV + c * (kBlk * 128), &tm_v, &v_full[0], c * 64, early * kBlk, g, b);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, C::kTmemCols);
@@ -276,6 +313,7 @@ __global__ void __launch_bounds__(128, 1)
         for (int c = 0; c < D / 64; ++c) tma_load_4d(dst + c * (kBlk * 128), map, full, c * 64, blk * kBlk, g, b);
       };
       int nk = 0, nv = 0, nq = 0;  // K, V and Q loads issued
+      if (*s_early) nk = nv = nq = 1;
       int kseg = 0, kq = 0, vseg = 0, vq = 0;
       bool stop = false;
       while (!stop && nv < total) {

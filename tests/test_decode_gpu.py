@@ -128,3 +128,21 @@ def test_decode_slot_ranges_over_many_rows_and_waves():
     rows = list(range(0, 1000, 7))
     ref_out, ref_lse = OD.decode_attention(q, k, v, sel, rows=rows)
     compare_attention(out[:, :, rows], lse[:, :, rows], ref_out, ref_lse)
+
+
+def test_decode_parts_starting_on_pads_duplicates_and_hidden_blocks():
+    """With explicit parts of 2 slots, every part's first slot decides whether
+    its first block is loaded before the list is deduplicated. Row 0's parts
+    start on a kept block, on a duplicate of an earlier slot, on a pad and on
+    a block after the row's position; row 1 starts on a pad and then on an
+    entry out of range (flagged and ignored)."""
+    q, k, v, sel = _inputs(12, 1, 4, 1, 2, 2000, 256, 8, pads=0, dups=0)
+    # 2000 keys: blocks 0-31; the rows sit at positions 1998 and 1999.
+    sel[0, 0, 0] = [3, 7, 3, 9, -1, 12, 31, 30]
+    sel[0, 0, 1] = [-1, 4, 32, 5, 5, 6, -1, -1]
+    clean = sel.copy()
+    clean[0, 0, 1, 2] = -1
+    for n_split in (4, 3):
+        out, lse, err = run(q, k, v, sel, n_split)
+        assert err & B.DEVERR_SEL
+        compare_attention(out, lse, *OD.decode_attention(q, k, v, clean))
