@@ -131,13 +131,15 @@ def test_decode_slot_ranges_over_many_rows_and_waves():
 
 
 def test_decode_parts_starting_on_pads_duplicates_and_hidden_blocks():
-    """With explicit parts of 2 slots, every part's first slot decides whether
-    its first block is loaded before the list is deduplicated. Row 0's parts
+    """Every part's first slot decides whether its first block is loaded
+    before the list is deduplicated. With 4 parts of 2 slots, row 0's parts
     start on a kept block, on a duplicate of an earlier slot, on a pad and on
-    a block after the row's position; row 1 starts on a pad and then on an
-    entry out of range (flagged and ignored)."""
-    q, k, v, sel = _inputs(12, 1, 4, 1, 2, 2000, 256, 8, pads=0, dups=0)
-    # 2000 keys: blocks 0-31; the rows sit at positions 1998 and 1999.
+    a block after the row's position; row 1's on a pad, on an entry out of
+    range (flagged and ignored), on a duplicate and on a pad. With 3 parts of
+    3 slots, two of them start on kept blocks that follow other entries."""
+    q, k, v, sel = _inputs(12, 1, 4, 1, 40, 2000, 256, 8, pads=0, dups=0)
+    # 2000 keys: blocks 0-31; rows 0 and 1 sit at positions 1960 and 1961, so
+    # block 31 (keys 1984-1999) is after both.
     sel[0, 0, 0] = [3, 7, 3, 9, -1, 12, 31, 30]
     sel[0, 0, 1] = [-1, 4, 32, 5, 5, 6, -1, -1]
     clean = sel.copy()
