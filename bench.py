@@ -78,7 +78,7 @@ BWD_NCU_TRAFFIC = {
 # The same for the decode kernel (mfa_decode_kernel) of --pass decode.
 DEC_KERNEL_SOURCES = ("mask_aware_block_mfa_b200/csrc/decode_sm100.cu", "mask_aware_block_mfa_b200/csrc/mfa_device.cuh")
 DEC_NCU_TRAFFIC = {
-    "decode_sel64k": (137_548_544, "0f12f154345792bb"),
+    "decode_sel64k": (137_655_552, "cbc2580e69c2360a"),
 }
 
 
